@@ -1,0 +1,243 @@
+// C ABI of the library (declared in include/bsa.h): argument validation,
+// workspace carve-up and the launch sequences of the three calls.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "bsa.h"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+thread_local char g_last_error[512] = {0};
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+bsa_status fail(bsa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+bsa_status fail(bsa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxN = kBlockK * kMaxKb;  // 131072
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bsa_status check_shape(const bsa_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.N < 1)
+    return fail(BSA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got B=%d H=%d N=%d)", s.B, s.H, s.N);
+  if (s.d != 64 && s.d != 128) return fail(BSA_ERR_INVALID_ARG, "d must be 64 or 128 (got %d)", s.d);
+  if (s.N > kMaxN) return fail(BSA_ERR_INVALID_ARG, "N must be <= %d (got %d)", kMaxN, s.N);
+  if (static_cast<int64_t>(s.B) * s.H > 65535)
+    return fail(BSA_ERR_INVALID_ARG, "B*H must be <= 65535 (got %lld)",
+                static_cast<long long>(s.B) * s.H);
+  return BSA_OK;
+}
+
+bsa_status check_tensor(const void* p, const char* name) {
+  if (p == nullptr) return fail(BSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return BSA_OK;
+}
+
+bsa_status check_ws(const bsa_shape& s, void* ws, size_t ws_bytes, Workspace* out) {
+  if (ws == nullptr) return fail(BSA_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(ws, 256)) return fail(BSA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t need = workspace_layout(s.B, s.H, s.N, s.d, out, ws);
+  if (ws_bytes < need)
+    return fail(BSA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  return BSA_OK;
+}
+
+bsa_status check_topk(float topk) {
+  if (!(topk > 0.f) || !(topk <= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "topk must lie in (0, 1] (got %g)", static_cast<double>(topk));
+  return BSA_OK;
+}
+
+int keep_count(float topk, int Kb) {
+  const double t = static_cast<double>(topk);
+  long long k = static_cast<long long>(ceil(t * static_cast<double>(Kb)));
+  if (k < 1) k = 1;
+  if (k > Kb) k = Kb;
+  return static_cast<int>(k);
+}
+
+#define BSA_TRY(x)                          \
+  do {                                      \
+    bsa_status _s = (x);                    \
+    if (_s != BSA_OK) return _s;            \
+  } while (0)
+
+#define BSA_CUDA(x, what)                   \
+  do {                                      \
+    cudaError_t _e = (x);                   \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base) {
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t Qb = (static_cast<size_t>(N) + kBlockQ - 1) / kBlockQ;
+  const size_t Kb = (static_cast<size_t>(N) + kBlockK - 1) / kBlockK;
+  size_t off = 0;
+  const size_t o_status = off; off = align256(off + sizeof(DeviceStatus));
+  const size_t o_qbar = off;   off = align256(off + BH * Qb * d * sizeof(float));
+  const size_t o_kbar = off;   off = align256(off + BH * Kb * d * sizeof(float));
+  const size_t o_idx = off;    off = align256(off + BH * Qb * Kb * sizeof(int16_t));
+  const size_t o_cnt = off;    off = align256(off + BH * Qb * sizeof(int32_t));
+  if (ws != nullptr) {
+    char* b = static_cast<char*>(base);
+    ws->status = reinterpret_cast<DeviceStatus*>(b + o_status);
+    ws->qbar = reinterpret_cast<float*>(b + o_qbar);
+    ws->kbar = reinterpret_cast<float*>(b + o_kbar);
+    ws->idx = reinterpret_cast<int16_t*>(b + o_idx);
+    ws->cnt = reinterpret_cast<int32_t*>(b + o_cnt);
+    ws->bytes = off;
+  }
+  return off;
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int bsa_abi_version(void) { return 1; }
+
+const char* bsa_status_string(bsa_status s) {
+  switch (s) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+  }
+  return "BSA_UNKNOWN_STATUS";
+}
+
+const char* bsa_last_error_message(void) { return g_last_error; }
+
+void bsa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000 ? 1000 : ns); }
+
+size_t bsa_workspace_bytes(bsa_shape s) {
+  if (check_shape(s) != BSA_OK) return 0;
+  return workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr);
+}
+
+bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, float* p_out,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  if (p_out == nullptr || !aligned(p_out, 4))
+    return fail(BSA_ERR_INVALID_ARG, "p_out is NULL or not 4-byte aligned");
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
+  BSA_CUDA(launch_block_scores(w.qbar, w.kbar, BH, s.N, s.d, p_out, st), "block-score kernel launch");
+  return BSA_OK;
+}
+
+bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk,
+                              uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  BSA_TRY(check_topk(topk));
+  if (mask_out == nullptr) return fail(BSA_ERR_INVALID_ARG, "mask_out is NULL");
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  const int Kb = (s.N + kBlockK - 1) / kBlockK;
+  BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
+  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), mask_out, w.idx, w.cnt, st),
+           "select kernel launch");
+  return BSA_OK;
+}
+
+bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bsa_shape s,
+                                 const uint8_t* mask_id, int is_causal, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  if (is_causal != 0) return fail(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  BSA_TRY(check_tensor(v, "v"));
+  BSA_TRY(check_tensor(out, "out"));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+  BSA_CUDA(launch_compact(mask_id, BH, s.N, w.idx, w.cnt, st), "compaction kernel launch");
+  const char* why = nullptr;
+  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status,
+                                   g_timeout_ns.load(), st, &why);
+  if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
+  return BSA_OK;
+}
+
+bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_shape s, float topk,
+                            int is_causal, void* out, uint8_t* mask_out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  if (is_causal != 0) return fail(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  BSA_TRY(check_tensor(v, "v"));
+  BSA_TRY(check_tensor(out, "out"));
+  BSA_TRY(check_topk(topk));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  const int Kb = (s.N + kBlockK - 1) / kBlockK;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+  BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
+  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), mask_out, w.idx, w.cnt, st),
+           "select kernel launch");
+  const char* why = nullptr;
+  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status,
+                                   g_timeout_ns.load(), st, &why);
+  if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
+  return BSA_OK;
+}
+
+bsa_status bsa_last_device_status(const void* ws, void* stream) {
+  g_last_error[0] = 0;
+  if (ws == nullptr || !aligned(ws, 256)) return fail(BSA_ERR_INVALID_ARG, "workspace is NULL or unaligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  BSA_CUDA(cudaStreamSynchronize(st), "stream synchronize");
+  DeviceStatus h;
+  BSA_CUDA(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost), "status read");
+  if (h.code == kDevTimeout)
+    return fail(BSA_ERR_TIMEOUT, "a bounded wait ran out (site %u, CTA %u)", h.where, h.block);
+  if (h.code != 0) return fail(BSA_ERR_CUDA, "unknown device status %u", h.code);
+  return BSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Host-side launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "bsa_common.cuh"
+
+namespace bsa {
+
+// Workspace carve-up (every section 256-byte aligned).
+struct Workspace {
+  DeviceStatus* status;  // 256 bytes
+  float* qbar;           // [B*H, Qb, d]
+  float* kbar;           // [B*H, Kb, d]
+  int16_t* idx;          // [B*H, Qb, Kb]  ascending kept key-block indices (prefix of cnt)
+  int32_t* cnt;          // [B*H, Qb]
+  size_t bytes;
+};
+
+size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base);
+
+// (a1, a2) mean-pool q over 128-row blocks and k over 64-row blocks.
+cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, float* qbar,
+                        float* kbar, cudaStream_t st);
+
+// (a3, a4) block scores and top-k; writes mask (optional), idx and cnt.
+cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, int d, int kkeep,
+                          uint8_t* mask_out, int16_t* idx, int32_t* cnt, cudaStream_t st);
+
+// (a3) block-score map only: p_out = softmax of the scaled block scores.
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, int N, int d,
+                                float* p_out, cudaStream_t st);
+
+// (a4') caller mask (NULL = all ones) -> idx and cnt.
+cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int16_t* idx, int32_t* cnt,
+                           cudaStream_t st);
+
+// (a5, a6) block-sparse attention forward over the idx lists.
+cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, int BH, int N,
+                             int d, const int16_t* idx, const int32_t* cnt, DeviceStatus* status,
+                             uint64_t timeout_ns, cudaStream_t st, const char** why);
+
+}  // namespace bsa

@@ -1,0 +1,370 @@
+// Selection stage: mean pooling of q/k, compressed block scores, top-k key
+// blocks per query block (radix select, ties to the lower block index), and
+// compaction of a caller mask into per-row kept-block index lists.
+//
+// Method: "SpargeAttention Documentation" -- spas_sage2_attn_meansim_topk_cuda
+// ("meansim", "topk") and the 128 x 64 mask of its "Mask Requirements".  All of
+// this is HBM-bound: q and k are read once with 16-byte loads, everything else
+// is small.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+// ------------------------------------------------------------------ pooling
+// One CTA per (query block i, head bh).  Thread (g, c) owns the 16-byte column
+// chunk c (8 bf16) of rows g, g + RG, ...; partial sums are combined in shared
+// memory in a fixed order, then divided by the number of valid rows.
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                   const __nv_bfloat16* __restrict__ k,
+                                                   float* __restrict__ qbar,
+                                                   float* __restrict__ kbar, int N, int Qb,
+                                                   int Kb) {
+  constexpr int TPR = D / 8;       // threads per row: one 16-byte chunk each
+  constexpr int RG = 256 / TPR;    // row groups
+  constexpr int RPT = 128 / RG;    // rows per thread within the 128-row block
+  static_assert(64 % RG == 0, "row groups must split at the 64-row boundary");
+  __shared__ float red[3][RG][D];  // partial sums: q, k (rows 0-63), k (rows 64-127)
+
+  const int i = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int t = threadIdx.x;
+  const int c = t % TPR;
+  const int g = t / TPR;
+  const int rows = min(kBlockQ, N - i * kBlockQ);
+  const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * kBlockQ) * D;
+  const uint4* q4 = reinterpret_cast<const uint4*>(q + base);
+  const uint4* k4 = reinterpret_cast<const uint4*>(k + base);
+
+  uint4 qv[RPT], kv[RPT];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const int r = g + RG * m;
+    if (r < rows) {
+      qv[m] = __ldg(q4 + static_cast<size_t>(r) * TPR + c);
+      kv[m] = __ldg(k4 + static_cast<size_t>(r) * TPR + c);
+    } else {
+      qv[m] = make_uint4(0, 0, 0, 0);
+      kv[m] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  float aq[8], ak0[8], ak1[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) aq[e] = ak0[e] = ak1[e] = 0.f;
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv[m]);
+    const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv[m]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 qf = __bfloat1622float2(qh[e]);
+      const float2 kf = __bfloat1622float2(kh[e]);
+      aq[2 * e] += qf.x;
+      aq[2 * e + 1] += qf.y;
+      if (m < RPT / 2) {
+        ak0[2 * e] += kf.x;
+        ak0[2 * e + 1] += kf.y;
+      } else {
+        ak1[2 * e] += kf.x;
+        ak1[2 * e + 1] += kf.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red[0][g][c * 8 + e] = aq[e];
+    red[1][g][c * 8 + e] = ak0[e];
+    red[2][g][c * 8 + e] = ak1[e];
+  }
+  __syncthreads();
+  const int rows_k0 = min(kBlockK, rows);
+  const int rows_k1 = rows - kBlockK;  // > 0 only if key block 2i+1 exists
+  for (int col = t; col < 3 * D; col += 256) {
+    const int which = col / D;
+    const int cc = col % D;
+    if (which == 2 && rows_k1 <= 0) continue;
+    float s = 0.f;
+#pragma unroll 8
+    for (int gg = 0; gg < RG; ++gg) s += red[which][gg][cc];
+    if (which == 0) {
+      qbar[(static_cast<size_t>(bh) * Qb + i) * D + cc] = s / static_cast<float>(rows);
+    } else if (which == 1) {
+      kbar[(static_cast<size_t>(bh) * Kb + 2 * i) * D + cc] = s / static_cast<float>(rows_k0);
+    } else {
+      kbar[(static_cast<size_t>(bh) * Kb + 2 * i + 1) * D + cc] = s / static_cast<float>(rows_k1);
+    }
+  }
+}
+
+// ------------------------------------------------------------ block scores
+constexpr int kSelG = 16;          // query blocks per CTA (one warp each)
+constexpr int kSelThreads = 512;
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key).
+// +0 and -0 map to the same key.
+__device__ __forceinline__ uint32_t float_key(float f) {
+  uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Dot products Qbar_i . Kbar_j for kSelG query blocks and every key block,
+// accumulated in fp32 in ascending d order, into sc[g][j].
+template <int D>
+__device__ __forceinline__ void block_dots(const float* __restrict__ qbar,
+                                           const float* __restrict__ kbar, int bh, int i0,
+                                           int Qb, int Kb, float* sq, float* sc) {
+  for (int e = threadIdx.x; e < kSelG * D; e += kSelThreads) {
+    const int g = e / D;
+    const int i = i0 + g;
+    sq[e] = (i < Qb) ? qbar[(static_cast<size_t>(bh) * Qb + i) * D + (e % D)] : 0.f;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < Kb; j += kSelThreads) {
+    const float4* kr = reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j) * D);
+    float acc[kSelG];
+#pragma unroll
+    for (int g = 0; g < kSelG; ++g) acc[g] = 0.f;
+#pragma unroll 4
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 kv = __ldg(kr + d4);
+#pragma unroll
+      for (int g = 0; g < kSelG; ++g) {
+        const float4 qv = reinterpret_cast<const float4*>(sq + g * D)[d4];
+        acc[g] = fmaf(qv.x, kv.x, acc[g]);
+        acc[g] = fmaf(qv.y, kv.y, acc[g]);
+        acc[g] = fmaf(qv.z, kv.z, acc[g]);
+        acc[g] = fmaf(qv.w, kv.w, acc[g]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kSelG; ++g) sc[g * Kb + j] = acc[g];
+  }
+  __syncthreads();
+}
+
+// Top-k of one row of dot products by one warp: a most-significant-digit radix
+// select over the float keys finds the kk-th largest key T and how many of the
+// keys equal to T are kept; the row is then emitted in ascending block order
+// (keys above T, plus the first `need_eq` keys equal to T).
+__device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, uint8_t* mask_row,
+                              int16_t* idx_row, int32_t* cnt_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = kk;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < Kb; j += 32) {
+      const uint32_t u = float_key(row[j]);
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // Lane l owns buckets 255-8l ... 248-8l (descending).
+    uint32_t cntb[8];
+    uint32_t local = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      cntb[t] = hist[255 - 8 * lane - t];
+      local += cntb[t];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= static_cast<uint32_t>(remaining));
+    const int src = __ffs(hit) - 1;  // first lane whose running count reaches `remaining`
+    uint32_t bucket = 0, above = 0;
+    if (lane == src) {
+      uint32_t run = incl - local;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (run + cntb[t] >= static_cast<uint32_t>(remaining)) {
+          bucket = 255 - 8 * lane - t;
+          above = run;
+          break;
+        }
+        run += cntb[t];
+      }
+    }
+    bucket = __shfl_sync(0xffffffffu, bucket, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    remaining -= static_cast<int>(above);
+    prefix |= bucket << shift;
+    pmask |= 255u << shift;
+    __syncwarp();
+  }
+  const uint32_t T = prefix;
+  const int need_eq = remaining;  // keys equal to T still to keep, lowest index first
+  int eq_seen = 0, kept = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < Kb; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = (j < Kb) ? float_key(row[j]) : 0u;
+    const bool eq = (j < Kb) && (u == T);
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool keep = (j < Kb) && (u > T || (eq && eq_seen + __popc(eqb & lt) < need_eq));
+    eq_seen += __popc(eqb);
+    const unsigned kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) idx_row[kept + __popc(kb & lt)] = static_cast<int16_t>(j);
+    if (mask_row != nullptr && j < Kb) mask_row[j] = keep ? 1 : 0;
+    kept += __popc(kb);
+  }
+  if (lane == 0) *cnt_out = kept;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ qbar,
+                                                             const float* __restrict__ kbar,
+                                                             int Qb, int Kb, int kk,
+                                                             uint8_t* __restrict__ mask_out,
+                                                             int16_t* __restrict__ idx,
+                                                             int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(16) float smem[];
+  float* sq = smem;                              // [kSelG][D]
+  float* sc = sq + kSelG * D;                    // [kSelG][Kb]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sc + kSelG * Kb);  // [16][256]
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * kSelG;
+  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
+  const int w = threadIdx.x >> 5;
+  const int i = i0 + w;
+  if (i >= Qb) return;
+  const size_t row = static_cast<size_t>(bh) * Qb + i;
+  warp_topk_row(sc + w * Kb, Kb, kk, hist + w * 256,
+                mask_out ? mask_out + row * Kb : nullptr, idx + row * Kb, cnt + row);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) block_scores_kernel(const float* __restrict__ qbar,
+                                                                   const float* __restrict__ kbar,
+                                                                   int Qb, int Kb, float scale,
+                                                                   float* __restrict__ p_out) {
+  extern __shared__ __align__(16) float smem[];
+  float* sq = smem;
+  float* sc = sq + kSelG * D;
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * kSelG;
+  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
+  const int w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int i = i0 + w;
+  if (i >= Qb) return;
+  const float* r = sc + w * Kb;
+  float mx = -INFINITY;
+  for (int j = lane; j < Kb; j += 32) mx = fmaxf(mx, r[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  for (int j = lane; j < Kb; j += 32) sum += expf((r[j] - mx) * scale);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = 1.f / sum;
+  float* out = p_out + (static_cast<size_t>(bh) * Qb + i) * Kb;
+  for (int j = lane; j < Kb; j += 32) out[j] = expf((r[j] - mx) * scale) * inv;
+}
+
+// ----------------------------------------------------------------- compaction
+// One warp per (b, h, i) row: kept block indices in ascending order.
+__global__ void __launch_bounds__(256) compact_kernel(const uint8_t* __restrict__ mask, int rows,
+                                                      int Kb, int16_t* __restrict__ idx,
+                                                      int32_t* __restrict__ cnt) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint8_t* m = mask ? mask + static_cast<size_t>(row) * Kb : nullptr;
+  int16_t* out = idx + static_cast<size_t>(row) * Kb;
+  const unsigned lt = (1u << lane) - 1u;
+  int kept = 0;
+  for (int base = 0; base < Kb; base += 32) {
+    const int j = base + lane;
+    const bool keep = (j < Kb) && (m == nullptr || m[j] != 0);
+    const unsigned b = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[kept + __popc(b & lt)] = static_cast<int16_t>(j);
+    kept += __popc(b);
+  }
+  if (lane == 0) cnt[row] = kept;
+}
+
+size_t select_smem(int d, int Kb, bool with_hist) {
+  return sizeof(float) * (static_cast<size_t>(kSelG) * d + static_cast<size_t>(kSelG) * Kb) +
+         (with_hist ? sizeof(uint32_t) * 16 * 256 : 0);
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, float* qbar,
+                        float* kbar, cudaStream_t st) {
+  const int Qb = (N + kBlockQ - 1) / kBlockQ;
+  const int Kb = (N + kBlockK - 1) / kBlockK;
+  dim3 grid(Qb, BH);
+  if (d == 128)
+    pool_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                           static_cast<const __nv_bfloat16*>(k), qbar, kbar, N,
+                                           Qb, Kb);
+  else
+    pool_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                          static_cast<const __nv_bfloat16*>(k), qbar, kbar, N, Qb,
+                                          Kb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, int d, int kk,
+                          uint8_t* mask_out, int16_t* idx, int32_t* cnt, cudaStream_t st) {
+  const int Qb = (N + kBlockQ - 1) / kBlockQ;
+  const int Kb = (N + kBlockK - 1) / kBlockK;
+  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
+  const size_t smem = select_smem(d, Kb, true);
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    select_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, mask_out, idx, cnt);
+  } else {
+    e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    select_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, mask_out, idx, cnt);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, int N, int d,
+                                float* p_out, cudaStream_t st) {
+  const int Qb = (N + kBlockQ - 1) / kBlockQ;
+  const int Kb = (N + kBlockK - 1) / kBlockK;
+  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
+  const size_t smem = select_smem(d, Kb, false);
+  const float scale = 1.0f / sqrtf(static_cast<float>(d));
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(block_scores_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    block_scores_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, p_out);
+  } else {
+    e = cudaFuncSetAttribute(block_scores_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    block_scores_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, p_out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int16_t* idx, int32_t* cnt,
+                           cudaStream_t st) {
+  const int Qb = (N + kBlockQ - 1) / kBlockQ;
+  const int Kb = (N + kBlockK - 1) / kBlockK;
+  const int rows = BH * Qb;
+  compact_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mask, rows, Kb, idx, cnt);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,125 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse attention library.
+ *
+ * Training-free, mean-pooled top-k block-sparse self-attention on a fixed
+ * 128 (query rows) x 64 (key rows) block grid, in two stages:
+ *
+ *   (1) selection: mean-pool q over 128-row blocks and k over 64-row blocks,
+ *       score the blocks with softmax(Qbar Kbar^T / sqrt(d)) per head, and keep
+ *       the top-k fraction of key blocks for every query block;
+ *   (2) attention: non-causal softmax attention that visits only the kept
+ *       128 x 64 tiles.
+ *
+ * The calls mirror the interface on "SpargeAttention Documentation":
+ * spas_sage2_attn_meansim_topk_cuda(q, k, v, topk, is_causal) (recommended API
+ * paragraph) and block_sparse_sage2_attn_cuda(q, k, v, mask_id) with the mask
+ * rules of its "Mask Requirements" section; the split into a selection call and
+ * an apply call follows build_plan / apply_plan on the AB-Attention README
+ * ("Use an existing pipeline", Q/K/V API).
+ *
+ * Conventions shared by every call
+ *  - q, k, v, out: device pointers to contiguous bf16 tensors of shape
+ *    [B, H, N, d] (row-major, d fastest), 16-byte aligned.  d is 64 or 128.
+ *  - Qb = ceil(N / 128), Kb = ceil(N / 64).  N <= 131072, so Kb <= 2048.
+ *  - mask tensors are uint8 [B, H, Qb, Kb], row-major; nonzero means "keep".
+ *  - ws: a device workspace of at least bsa_workspace_bytes(shape) bytes,
+ *    256-byte aligned, owned by the caller.  The library never allocates and
+ *    keeps no per-call state between calls; calls that share one workspace must
+ *    be ordered on one stream.
+ *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on it and returns after launching.
+ *  - The attention scale is 1/sqrt(d), as in scaled-dot-product attention.
+ *  - Errors: arguments are validated on the host before anything is launched;
+ *    a rejected call returns BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED and
+ *    touches no memory.  A failed launch returns BSA_ERR_CUDA.  Every wait
+ *    inside the attention kernel is bounded in time; if one runs out the kernel
+ *    records it in ws and returns early, which bsa_last_device_status reports
+ *    as BSA_ERR_TIMEOUT.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment, topk or workspace size */
+  BSA_ERR_UNSUPPORTED = 2, /* is_causal != 0 */
+  BSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  BSA_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out */
+} bsa_status;
+
+typedef struct {
+  int32_t B; /* batch */
+  int32_t H; /* heads */
+  int32_t N; /* sequence length (tokens) */
+  int32_t d; /* head dimension: 64 or 128 */
+} bsa_shape;
+
+/* Version of this ABI (incremented on incompatible changes). */
+int bsa_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* bsa_status_string(bsa_status s);
+
+/* Detail of the last host-side rejection or CUDA error on the calling thread
+ * (static, thread-local string; empty if none). */
+const char* bsa_last_error_message(void);
+
+/* Workspace bytes needed for a shape: pooled means, the compacted per-query-
+ * block key-block index list, its counts and the device status word.  Returns 0
+ * for a shape the library rejects. */
+size_t bsa_workspace_bytes(bsa_shape s);
+
+/* Compressed block-score map.  Writes p_out, fp32 [B, H, Qb, Kb] (device),
+ * with p_out[b,h,i,:] = softmax_j(Qbar_i . Kbar_j / sqrt(d)), where Qbar_i is
+ * the mean of q rows [128 i, min(128 i + 128, N)) and Kbar_j the mean of k rows
+ * [64 j, min(64 j + 64, N)) (means over valid rows only).  This is the score
+ * that the top-k selection ranks. */
+bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, float* p_out,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* Selection stage.  Writes mask_out (device, uint8 [B, H, Qb, Kb]) with exactly
+ * kk = clamp(ceil(topk * Kb), 1, Kb) ones per (b, h, i) row: the kk key blocks
+ * with the largest block score, equal scores going to the lower block index.
+ * kk is evaluated in double precision on the float value of topk.
+ * topk must lie in (0, 1]. */
+bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk,
+                              uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Attention over caller-chosen tiles.  mask_id (device, uint8 [B, H, Qb, Kb];
+ * NULL means all ones, i.e. dense attention) selects the kept 128 x 64 tiles.
+ * For every query row r of block i: out[r] = sum over kept tiles j and key rows
+ * c < N of block j of softmax_c(q_r . k_c / sqrt(d)) v_c, the softmax taken
+ * over the union of the kept keys.  A query block that keeps no key block gets
+ * an all-zero output.  Rows >= N are never written.  is_causal must be 0. */
+bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bsa_shape s,
+                                 const uint8_t* mask_id, int is_causal, void* out,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Selection followed by attention in one call (three kernels on one stream,
+ * no host synchronisation).  mask_out is optional (NULL: not written); when
+ * given it receives the selection mask of sparse_attn_select. */
+bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_shape s, float topk,
+                            int is_causal, void* out, uint8_t* mask_out, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reports what the kernels of the last call that
+ * used `ws` recorded: BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out), or
+ * BSA_ERR_CUDA if the stream holds an error. */
+bsa_status bsa_last_device_status(const void* ws, void* stream);
+
+/* Limit of every bounded wait inside the kernels, in nanoseconds (process-wide;
+ * default 2e9).  Values below 1000 are raised to 1000. */
+void bsa_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -91,7 +91,7 @@ def pool_mean(x: np.ndarray, block: int) -> np.ndarray:
 def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
     """P = softmax_j(Qbar_i . Kbar_j / sqrt(d)) per (b, h, i) -> [B, H, Qb, Kb]."""
     d = qbar.shape[-1]
-    S = np.einsum("bhid,bhjd->bhij", qbar, kbar) / math.sqrt(d)
+    S = np.matmul(qbar, np.swapaxes(kbar, -1, -2)) / math.sqrt(d)
     S = S - S.max(axis=-1, keepdims=True)
     E = np.exp(S)
     return E / E.sum(axis=-1, keepdims=True)

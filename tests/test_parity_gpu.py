@@ -1,0 +1,165 @@
+"""GPU parity against the fp64 oracle on small and ragged shapes, through the C ABI
+(via the Python binding), plus edge cases: empty rows, single tiles, odd kept
+counts, ragged last blocks, the dense limit, compaction exactness, output canary
+and determinism."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_14_b200 as bsa
+from block_sparse_attention_14_b200 import workloads as W
+from oracle import bsa_oracle as O
+from tests.parity import assert_close, compare_masks
+
+pytestmark = pytest.mark.gpu
+
+
+def _qkv(B, H, N, d, seed, scale=1.0):
+    """q, k ~ N(0, scale^2) (a larger scale sharpens the softmax); v ~ N(0, 1) as in
+    the workloads, so |out| stays where a 2e-2 absolute bound is meaningful for bf16."""
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn(B, H, N, d, generator=g) for _ in range(3))
+    return [(q * scale).to(torch.bfloat16), (k * scale).to(torch.bfloat16), v.to(torch.bfloat16)]
+
+
+def _cuda(*ts):
+    return [t.cuda() for t in ts]
+
+
+SHAPES = [(1, 2, 1024, 64), (1, 2, 1024, 128), (2, 3, 300, 64), (1, 2, 300, 128),
+          (1, 1, 1, 64), (1, 1, 65, 128), (1, 2, 4113, 128), (1, 1, 2000, 64)]
+
+
+@pytest.mark.parametrize("B,H,N,d", SHAPES)
+def test_dense_mask_none_matches_oracle(B, H, N, d, cuda_device):
+    q, k, v = _qkv(B, H, N, d, seed=N + d, scale=1.5)
+    out = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), None)
+    torch.cuda.synchronize()
+    ref = O.dense_attention(q, k, v)
+    assert_close(out.float().cpu().numpy(), ref, f"dense {B,H,N,d}")
+
+
+@pytest.mark.parametrize("B,H,N,d,density", [(1, 3, 1000, 64, 0.3), (1, 3, 1000, 128, 0.3),
+                                             (2, 2, 2081, 128, 0.5), (1, 2, 4096, 64, 0.1),
+                                             (1, 2, 1537, 128, 0.05)])
+def test_caller_mask_matches_oracle(B, H, N, d, density, cuda_device):
+    q, k, v = _qkv(B, H, N, d, seed=7 * N + d, scale=2.0)
+    Qb, Kb = O.block_counts(N)
+    g = torch.Generator().manual_seed(N)
+    mask = (torch.rand(B, H, Qb, Kb, generator=g) < density).to(torch.uint8)
+    mask[0, 0, 0] = 0                  # empty row -> zero output
+    mask[0, -1, -1] = 0
+    mask[0, -1, -1, -1] = 1            # only the ragged last key block
+    if Qb > 1:
+        mask[0, 0, 1] = 0
+        mask[0, 0, 1, Kb // 2] = 1     # a single kept tile (odd count)
+        mask[-1, 0, 1] = 1             # a full row (dense)
+    out = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), mask.cuda())
+    torch.cuda.synchronize()
+    ref = O.block_sparse_attention(q, k, v, mask.numpy())
+    got = out.float().cpu().numpy()
+    assert np.all(got[0, 0, :128] == 0), "empty row must be exactly zero"
+    assert_close(got, ref, f"mask {B,H,N,d,density}")
+
+
+def test_tiny_workload_fused_topk(cuda_device):
+    wl = W.WORKLOADS["tiny"]
+    q, k, v = W.make_qkv(wl)
+    out, mask = bsa.sparse_attn_topk(*_cuda(q, k, v), topk=0.5, return_mask=True)
+    torch.cuda.synchronize()
+    mref, P = O.select(q, k, 0.5)
+    kk = O.keep_count(0.5, wl.Kb)
+    bad, n_ex, _ = compare_masks(mask, mref, P, kk)
+    assert bad == 0
+    ref = O.block_sparse_attention(q, k, v, mref)
+    same = np.all(mask.cpu().numpy() == mref, axis=-1)  # compare rows whose masks agree
+    got = out.float().cpu().numpy()
+    rows = np.repeat(same, 128, axis=2)[:, :, :wl.N]
+    assert_close(got[rows], ref[rows], "tiny fused")
+
+
+@pytest.mark.parametrize("N,d,topk", [(3000, 128, 0.3), (3000, 64, 0.5), (777, 128, 0.2),
+                                      (8192, 128, 0.1), (5000, 64, 1.0)])
+def test_fused_topk_matches_oracle(N, d, topk, cuda_device):
+    wl = W.custom("c", B=1, H=3, d=d, N=N, seed=N)
+    q, k, v = W.make_qkv(wl)
+    out, mask = bsa.sparse_attn_topk(*_cuda(q, k, v), topk=topk, return_mask=True)
+    torch.cuda.synchronize()
+    mref, P = O.select(q, k, topk)
+    bad, _, diff_ex = compare_masks(mask, mref, P, O.keep_count(topk, wl.Kb))
+    assert bad == 0
+    ref = O.block_sparse_attention(q, k, v, mref)
+    same = np.all(mask.cpu().numpy() == mref, axis=-1)
+    rows = np.repeat(same, 128, axis=2)[:, :, :N]
+    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"fused {N,d,topk}")
+
+
+def test_select_equals_fused_mask_and_block_scores(cuda_device):
+    wl = W.custom("s", B=2, H=2, d=128, N=2500, seed=3)
+    q, k, v = _cuda(*W.make_qkv(wl))
+    m1 = bsa.sparse_attn_select(q, k, 0.4)
+    _, m2 = bsa.sparse_attn_topk(q, k, v, 0.4, return_mask=True)
+    assert torch.equal(m1, m2)
+    P = bsa.sparse_attn_block_scores(q, k)
+    torch.cuda.synchronize()
+    _, Pref = O.select(q.cpu(), k.cpu(), 0.4)
+    Pg = P.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(Pg.sum(-1), 1.0, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(Pg, Pref, rtol=1e-4, atol=1e-7)
+
+
+def test_topk_one_equals_dense_bitwise(cuda_device):
+    q, k, v = _cuda(*_qkv(1, 2, 3001, 128, seed=5))
+    a = bsa.sparse_attn_topk(q, k, v, 1.0)
+    b = bsa.block_sparse_attn_fwd(q, k, v, None)
+    ones = torch.ones(1, 2, *O.block_counts(3001), dtype=torch.uint8, device="cuda")
+    c = bsa.block_sparse_attn_fwd(q, k, v, ones)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(b, c)
+
+
+def test_compaction_is_exact(cuda_device):
+    B, H, N, d = 1, 4, 5000, 64
+    q, k, v = _cuda(*_qkv(B, H, N, d, seed=11))
+    Qb, Kb = O.block_counts(N)
+    g = torch.Generator().manual_seed(2)
+    mask = (torch.rand(B, H, Qb, Kb, generator=g) < 0.37).to(torch.uint8)
+    mask[0, 1, 3] = 7  # any nonzero value means keep
+    ws = bsa.make_workspace(B, H, N, d)
+    bsa.block_sparse_attn_fwd(q, k, v, mask.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    r = lambda x: (x + 255) // 256 * 256
+    BH = B * H
+    o_idx = 256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4)
+    o_cnt = o_idx + r(BH * Qb * Kb * 2)
+    idx = ws[o_idx:o_idx + BH * Qb * Kb * 2].view(torch.int16).view(BH * Qb, Kb).cpu().numpy()
+    cnt = ws[o_cnt:o_cnt + BH * Qb * 4].view(torch.int32).cpu().numpy()
+    m = mask.view(BH * Qb, Kb).numpy()
+    for row in range(BH * Qb):
+        want = np.flatnonzero(m[row])
+        assert cnt[row] == want.size
+        assert np.array_equal(idx[row, :cnt[row]], want)
+
+
+def test_no_writes_outside_output_and_deterministic(cuda_device):
+    B, H, N, d = 1, 3, 1111, 128
+    q, k, v = _cuda(*_qkv(B, H, N, d, seed=13))
+    n = B * H * N * d
+    buf = torch.full((n + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[:n].view(B, H, N, d)
+    bsa.sparse_attn_topk(q, k, v, 0.5, out=out)
+    first = out.clone()
+    bsa.sparse_attn_topk(q, k, v, 0.5, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(buf[n:] == 7.0)
+    assert torch.equal(first, out)
+
+
+def test_causal_rejected_and_status_ok(cuda_device):
+    q, k, v = _cuda(*_qkv(1, 1, 256, 64, seed=1))
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.sparse_attn_topk(q, k, v, 0.5, is_causal=True)
+    assert e.value.status == 2
+    ws = bsa.make_workspace(1, 1, 256, 64)
+    bsa.sparse_attn_topk(q, k, v, 0.5, workspace=ws)
+    bsa.last_device_status(ws)  # raises on a recorded timeout
