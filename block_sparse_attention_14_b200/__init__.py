@@ -31,7 +31,7 @@ import torch
 __all__ = [
     "BsaError", "sparse_attn_topk", "block_sparse_attn_fwd", "sparse_attn_select",
     "sparse_attn_block_scores", "workspace_bytes", "make_workspace", "last_device_status",
-    "set_wait_timeout_ns", "block_counts", "keep_count", "library_path", "lib",
+    "set_wait_timeout_ns", "block_sparse_attn_plan", "block_sparse_attn_apply", "block_counts", "keep_count", "library_path", "lib",
 ]
 
 BLOCK_Q = 128
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.block_sparse_attn_fwd.argtypes = [vp, vp, vp, Shape, vp, i32, vp, vp, sz, vp]
         L.sparse_attn_topk.restype = i32
         L.sparse_attn_topk.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp, sz, vp]
+        L.block_sparse_attn_plan.restype = i32
+        L.block_sparse_attn_plan.argtypes = [vp, Shape, vp, sz, vp]
+        L.block_sparse_attn_apply.restype = i32
+        L.block_sparse_attn_apply.argtypes = [vp, vp, vp, Shape, vp, vp, sz, vp]
         L.bsa_last_device_status.restype = i32
         L.bsa_last_device_status.argtypes = [vp, vp]
         L.bsa_set_wait_timeout_ns.restype = None
@@ -222,6 +226,28 @@ def sparse_attn_block_scores(q, k, *, out=None, workspace=None) -> torch.Tensor:
     ws, wp, wn = _ws(q, workspace)
     _check(lib().sparse_attn_block_scores(q.data_ptr(), k.data_ptr(), _shape_of(q), out.data_ptr(),
                                           wp, wn, _stream(q)))
+    return out
+
+
+def block_sparse_attn_plan(q, mask_id=None, *, workspace=None) -> torch.Tensor:
+    """Compact mask_id (None = dense) into a reusable plan held in the returned workspace."""
+    B, H, N, d = q.shape
+    m = _mask_arg(mask_id, q) if mask_id is not None else None
+    ws, wp, wn = _ws(q, workspace)
+    _check(lib().block_sparse_attn_plan(m.data_ptr() if m is not None else None, _shape_of(q), wp, wn,
+                                        _stream(q)))
+    return ws
+
+
+def block_sparse_attn_apply(q, k, v, workspace, *, out=None):
+    """Attention over the plan held in `workspace` (from sparse_attn_select,
+    sparse_attn_topk or block_sparse_attn_plan on the same shape)."""
+    _qkv(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    _qkv(q, out)
+    _check(lib().block_sparse_attn_apply(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q),
+                                         out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                         _stream(q)))
     return out
 
 

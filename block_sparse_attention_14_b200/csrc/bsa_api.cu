@@ -227,6 +227,36 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
   return BSA_OK;
 }
 
+bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  BSA_CUDA(launch_compact(mask_id, s.B * s.H, s.N, w.idx, w.cnt, st), "compaction kernel launch");
+  return BSA_OK;
+}
+
+bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, bsa_shape s,
+                                   void* out, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  BSA_TRY(check_tensor(v, "v"));
+  BSA_TRY(check_tensor(out, "out"));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+  const char* why = nullptr;
+  cudaError_t e = launch_attention(q, k, v, out, s.B * s.H, s.N, s.d, w.idx, w.cnt, w.status,
+                                   g_timeout_ns.load(), st, &why);
+  if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
+  return BSA_OK;
+}
+
 bsa_status bsa_last_device_status(const void* ws, void* stream) {
   g_last_error[0] = 0;
   if (ws == nullptr || !aligned(ws, 256)) return fail(BSA_ERR_INVALID_ARG, "workspace is NULL or unaligned");

@@ -109,6 +109,20 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
                             int is_causal, void* out, uint8_t* mask_out, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* Plan / apply split (the build_plan / apply_plan pattern of the AB-Attention
+ * README, "Use an existing pipeline"): the kept-block lists that
+ * sparse_attn_select, sparse_attn_topk or block_sparse_attn_plan leave in ws
+ * form a reusable plan.  block_sparse_attn_plan compacts a caller mask
+ * (NULL = all ones) into ws without running attention. */
+bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* Attention over the plan currently held in ws (see block_sparse_attn_plan);
+ * same output contract as block_sparse_attn_fwd.  The plan must have been
+ * made for the same shape; ws is not modified apart from its status word. */
+bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, bsa_shape s,
+                                   void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reports what the kernels of the last call that
  * used `ws` recorded: BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out), or
  * BSA_ERR_CUDA if the stream holds an error. */
