@@ -3,20 +3,28 @@
 // and its "Mask Requirements" ("SpargeAttention Documentation"): non-causal,
 // bf16 inputs, scale 1/sqrt(d).
 //
-// One CTA per (head, query block), 256 threads:
-//   warp 0      TMA producer for the Q tile and the kept K tiles
-//   warp 1      TMEM owner and MMA issuer (one thread issues tcgen05.mma)
-//   warp 2      TMA producer for the kept V tiles
-//   warps 4-7   softmax and epilogue; thread t owns query row t, which is TMEM
-//               lane t, so row max / row sum need no shuffles
-// Kept key blocks are consumed in pairs (128 keys), so S = Q K^T is one
-// M=128, N=128 tensor-core tile per pair (N=64 for an odd last block), and
-// O += P V runs with K=128.  S is double-buffered in TMEM so QK^T of pair j+1
-// overlaps the softmax of pair j.  P is written back to TMEM as bf16 (or to
-// shared memory in the kPInTmem=false variant) and O accumulates in TMEM.
+// One CTA per (head, query block), 384 threads in three warpgroups:
+//   WG0  warp 0: TMA producer for the Q tile and the kept K tiles
+//        warp 1: TMEM owner; one thread issues the Q K^T tcgen05.mma
+//        warp 2: TMA producer for the kept V tiles
+//        warp 3: one thread issues the P V tcgen05.mma
+//        (the two issuers touch disjoint TMEM -- S buffers vs O accumulators
+//        -- and synchronise only through the softmax barriers)
+//   WG1, WG2: softmax.  Kept key blocks are consumed in pairs (128 keys); WG1
+//        takes the even pairs and WG2 the odd ones.  Thread t of a softmax
+//        warpgroup owns query row t, which is TMEM lane t, so row max / row
+//        sum need no shuffles.
+// Per pair j, S = Q K^T is one M=128, N=128 tcgen05 tile (N=64 for an odd last
+// block) in the S buffer of warpgroup w = j % 2.  The warpgroup copies S into
+// registers and releases the buffer at once, so the tensor core computes
+// S_{j+2} while the exponentials of pair j run.  P (bf16) goes to a per-
+// warpgroup shared-memory tile in the K-major 128-byte-swizzled layout, and
+// O_w += P V accumulates in TMEM.  Each warpgroup keeps its own running max,
+// row sum and O accumulator; the two are merged in the epilogue.
 // The online softmax works in the exp2 domain and only rescales O when the row
 // maximum grows by more than 2^8, which keeps every exponent <= 2^8 and is
-// exact because l and O always share the same reference maximum.
+// exact because l and O always share the same reference maximum.  Half of the
+// exponentials run on the FMA pipes (exp2_poly2) and half on MUFU.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -29,6 +37,13 @@
 namespace bsa {
 namespace {
 
+// Column pairs c with bit (c % 8) set use the FMA-pipe exp2 polynomial; the
+// others use MUFU ex2.  Balances MUFU throughput against issue slots.
+#ifndef BSA_POLY_PATTERN
+#define BSA_POLY_PATTERN 0xAA
+#endif
+constexpr unsigned kPolyPattern = BSA_POLY_PATTERN;
+
 enum WaitSite : uint32_t {
   kWaitQ = 1,
   kWaitKFull = 2,
@@ -38,8 +53,8 @@ enum WaitSite : uint32_t {
   kWaitSFull = 6,
   kWaitPFull = 7,
   kWaitODone = 8,
-  kWaitFinal = 9,
-  kWaitDrain = 10,
+  kWaitSFree = 9,
+  kWaitPFree = 10,
 };
 
 struct AttnArgs {
@@ -52,38 +67,42 @@ struct AttnArgs {
   float scale_log2;  // log2(e) / sqrt(d)
 };
 
-template <int D, bool kPInTmem>
+template <int D>
 struct Cfg {
+  static constexpr int kThreads = 384;
   static constexpr int kChunk = 16384;           // one 128-row x 64-column bf16 SW128 chunk
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;   // a pair of 64-row key blocks
-  static constexpr int kKSt = (D == 128) ? 2 : (kPInTmem ? 4 : 3);
-  static constexpr int kVSt = (D == 128) ? (kPInTmem ? 3 : 2) : (kPInTmem ? 4 : 3);
-  static constexpr int kPBytes = kPInTmem ? 0 : 128 * 128 * 2;
+  static constexpr int kKSt = (D == 128) ? 2 : 3;
+  static constexpr int kVSt = (D == 128) ? 2 : 3;
+  static constexpr int kPBytes = 128 * 128 * 2;  // one warpgroup's P tile
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + kKSt * kKVBytes;
   static constexpr int kOffP = kOffV + kVSt * kKVBytes;
-  static constexpr int kSmem = kOffP + kPBytes + 1024;  // + alignment slack
-  // TMEM columns
-  static constexpr uint32_t kColS = 0;    // two 128-column S buffers
-  static constexpr uint32_t kColO = 256;  // D columns
-  static constexpr uint32_t kColP = 384;  // 64 columns of packed bf16 pairs
+  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;  // + alignment slack
+  // TMEM columns: S buffer w at 128 w, O_w at 256 + D w.
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColO = 256;
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t kRegCtl = 56;   // registers per thread, control warpgroup
+  static constexpr uint32_t kRegSm = 224;   // registers per thread, softmax warpgroups
+  static_assert(kSmem + 512 <= 227 * 1024, "shared memory budget (dynamic + static)");
   static_assert(kSmem > 114 * 1024, "one CTA per SM (it allocates all 512 TMEM columns)");
+  static_assert(128 * kRegCtl + 256 * kRegSm <= 168 * 384, "register split must fit the launch budget");
 };
 
-template <int D, bool kPInTmem>
-__global__ void __launch_bounds__(256, 1)
+template <int D>
+__global__ void __launch_bounds__(384, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  using C = Cfg<D, kPInTmem>;
+  using C = Cfg<D>;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_q, bar_kfull[C::kKSt], bar_kempty[C::kKSt],
-      bar_vfull[C::kVSt], bar_vempty[C::kVSt], bar_sfull[2], bar_pfull, bar_odone, bar_final;
+      bar_vfull[C::kVSt], bar_vempty[C::kVSt], bar_sfull[2], bar_sfree[2], bar_pfull[2],
+      bar_pfree[2], bar_odone, bar_qkdone;
   __shared__ uint32_t s_tmem;
-  __shared__ int16_t s_idx[kMaxKb];
+  __shared__ int s_cnt, s_last, s_fail;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -91,13 +110,17 @@ __global__ void __launch_bounds__(256, 1)
   const int qi = blockIdx.x - bh * a.Qb;
   const size_t row_id = static_cast<size_t>(bh) * a.Qb + qi;
   const int rows_valid = min(kBlockQ, a.N - qi * kBlockQ);
+  const int16_t* idx_row = a.idx + row_id * a.Kb;
   __nv_bfloat16* out_blk = a.out + (static_cast<size_t>(bh) * a.N + static_cast<size_t>(qi) * kBlockQ) * D;
 
   // One thread reads the count (and whether an earlier CTA already gave up) so
   // that every thread takes the same early-exit decision.
-  __shared__ int s_cnt;
-  if (threadIdx.x == 0)
-    s_cnt = (*reinterpret_cast<volatile uint32_t*>(&a.status->code) != 0) ? -1 : a.cnt[row_id];
+  if (threadIdx.x == 0) {
+    const int c = (*reinterpret_cast<volatile uint32_t*>(&a.status->code) != 0) ? -1 : a.cnt[row_id];
+    s_cnt = c;
+    s_last = c > 0 ? idx_row[c - 1] : -1;  // the ragged last key block can only be the last kept one
+    s_fail = 0;
+  }
   __syncthreads();
   const int cnt = s_cnt;
   if (cnt < 0) return;
@@ -106,13 +129,12 @@ __global__ void __launch_bounds__(256, 1)
     for (int e = threadIdx.x; e < rows_valid * D / 8; e += blockDim.x) o4[e] = make_uint4(0, 0, 0, 0);
     return;
   }
-  for (int t = threadIdx.x; t < cnt; t += blockDim.x) s_idx[t] = a.idx[row_id * a.Kb + t];
 
   const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
   const uint32_t sQ = base;
   const uint32_t sK0 = base + C::kOffK;
   const uint32_t sV0 = base + C::kOffV;
-  const uint32_t sP = base + C::kOffP;
+  const uint32_t sP0 = base + C::kOffP;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bar_q), 1);
@@ -124,11 +146,14 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(smem_u32(&bar_vfull[s]), 1);
       mbar_init(smem_u32(&bar_vempty[s]), 1);
     }
-    mbar_init(smem_u32(&bar_sfull[0]), 1);
-    mbar_init(smem_u32(&bar_sfull[1]), 1);
-    mbar_init(smem_u32(&bar_pfull), 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(smem_u32(&bar_sfull[w]), 1);
+      mbar_init(smem_u32(&bar_sfree[w]), 128);
+      mbar_init(smem_u32(&bar_pfull[w]), 128);
+      mbar_init(smem_u32(&bar_pfree[w]), 1);
+    }
     mbar_init(smem_u32(&bar_odone), 1);
-    mbar_init(smem_u32(&bar_final), 1);
+    mbar_init(smem_u32(&bar_qkdone), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -145,214 +170,265 @@ __global__ void __launch_bounds__(256, 1)
 
   // Stage-issue counters, used by the producers to drain in-flight copies.
   uint32_t issued[4] = {0, 0, 0, 0};
+  bool mma_issued = false;
 
-  if (warp == 0) {
-    // ------------------------------------------------ Q / K producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      mbar_expect_tx(smem_u32(&bar_q), C::kQBytes);
+  if (warp < 4) {
+    setmaxnreg_dec<C::kRegCtl>();
+    if ((warp == 0 || warp == 2) && lane == 0) {
+      // ---------------------------------------------- TMA producers
+      // warp 0: Q, then the K tiles of every pair; warp 2: the V tiles.
+      const bool is_k = warp == 0;
+      const int nst = is_k ? C::kKSt : C::kVSt;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      const uint32_t ring = is_k ? sK0 : sV0;
+      uint64_t* full = is_k ? bar_kfull : bar_vfull;
+      uint64_t* empty = is_k ? bar_kempty : bar_vempty;
+      tma_prefetch_desc(map);
+      if (is_k) {
+        tma_prefetch_desc(&tm_q);
+        mbar_expect_tx(smem_u32(&bar_q), C::kQBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(sQ + c * C::kChunk, &tm_q, smem_u32(&bar_q), c * 64, qi * kBlockQ, bh);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sQ + c * C::kChunk, &tm_q, smem_u32(&bar_q), c * 64, qi * kBlockQ, bh);
+      }
+      int b0 = __ldg(idx_row), b1 = cnt > 1 ? __ldg(idx_row + 1) : 0;
       for (int j = 0; j < npairs; ++j) {
-        const int s = j % C::kKSt;
-        const int n = j / C::kKSt;
-        if (n > 0 && !mbar_wait(smem_u32(&bar_kempty[s]), (n - 1) & 1, st, tmo, kWaitKEmpty)) break;
+        const int nx0 = 2 * j + 2 < cnt ? __ldg(idx_row + 2 * j + 2) : 0;  // next pair, prefetched
+        const int nx1 = 2 * j + 3 < cnt ? __ldg(idx_row + 2 * j + 3) : 0;
+        const int s = j % nst;
+        const int n = j / nst;
+        if (n > 0 && !mbar_wait(smem_u32(&empty[s]), (n - 1) & 1, st, tmo, is_k ? kWaitKEmpty : kWaitVEmpty)) break;
         const int nb = min(2, cnt - 2 * j);
-        const uint32_t bar = smem_u32(&bar_kfull[s]);
+        const uint32_t bar = smem_u32(&full[s]);
         mbar_expect_tx(bar, nb * 64 * D * 2);
-        for (int h = 0; h < nb; ++h) {
-          const int blk = s_idx[2 * j + h];
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(ring + s * C::kKVBytes + c * C::kChunk, map, bar, c * 64, b0 * kBlockK, bh);
+        if (nb == 2) {
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sK0 + s * C::kKVBytes + c * C::kChunk + h * 8192, &tm_k, bar, c * 64,
-                        blk * kBlockK, bh);
+            tma_load_3d(ring + s * C::kKVBytes + c * C::kChunk + 8192, map, bar, c * 64, b1 * kBlockK, bh);
         }
         ++issued[s];
+        b0 = nx0;
+        b1 = nx1;
       }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------ V producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_v);
-      for (int j = 0; j < npairs; ++j) {
-        const int s = j % C::kVSt;
-        const int n = j / C::kVSt;
-        if (n > 0 && !mbar_wait(smem_u32(&bar_vempty[s]), (n - 1) & 1, st, tmo, kWaitVEmpty)) break;
-        const int nb = min(2, cnt - 2 * j);
-        const uint32_t bar = smem_u32(&bar_vfull[s]);
-        mbar_expect_tx(bar, nb * 64 * D * 2);
-        for (int h = 0; h < nb; ++h) {
-          const int blk = s_idx[2 * j + h];
-#pragma unroll
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sV0 + s * C::kKVBytes + c * C::kChunk + h * 8192, &tm_v, bar, c * 64,
-                        blk * kBlockK, bh);
-        }
-        ++issued[s];
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_pv = idesc_bf16(128, D, true);
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------- QK^T issuer
+      // S_j = Q K_j^T into S buffer j % 2, once the softmax has copied S_{j-2}
+      // out of that buffer.
+      const uint64_t qd = sw128_desc(sQ, 16, 1024);
       bool ok = mbar_wait(smem_u32(&bar_q), 0, st, tmo, kWaitQ);
-      tc_fence_after();
-      auto issue_qk = [&](int j) -> bool {
+      mma_issued = true;
+      for (int j = 0; ok && j < npairs; ++j) {
+        const int w = j & 1;
+        if (j >= 2 && !(ok = mbar_wait(smem_u32(&bar_sfree[w]), ((j - 2) >> 1) & 1, st, tmo, kWaitSFree))) break;
         const int s = j % C::kKSt;
-        if (!mbar_wait(smem_u32(&bar_kfull[s]), (j / C::kKSt) & 1, st, tmo, kWaitKFull)) return false;
+        if (!(ok = mbar_wait(smem_u32(&bar_kfull[s]), (j / C::kKSt) & 1, st, tmo, kWaitKFull))) break;
         tc_fence_after();
         const int nb = min(2, cnt - 2 * j);
         const uint32_t idesc = idesc_bf16(128, 64 * nb, false);
-        const uint32_t dt = tmem + C::kColS + (j & 1) * 128;
-        const uint32_t kb = sK0 + s * C::kKVBytes;
+        const uint32_t dt = tmem + C::kColS + w * 128;
+        const uint64_t kd = sw128_desc(sK0 + s * C::kKVBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunk + (kk & 3) * 32;
-          umma_ss(dt, sw128_desc(sQ + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc, kk > 0);
+          // descriptor start addresses advance in 16-byte units
+          const uint32_t off = ((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4;
+          umma_ss(dt, qd + off, kd + off, idesc, kk > 0);
         }
-        umma_commit(smem_u32(&bar_sfull[j & 1]));
+        umma_commit(smem_u32(&bar_sfull[w]));
         umma_commit(smem_u32(&bar_kempty[s]));
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
+      }
+      umma_commit(smem_u32(&bar_qkdone));
+    } else if (warp == 3 && lane == 0) {
+      // ---------------------------------------------- P.V issuer
+      // O_w += P_j V_j (w = j % 2) once P_j is in shared memory.
+      const uint32_t idesc_pv = idesc_bf16(128, D, true);
+      bool ok = true;
+      mma_issued = true;
       for (int j = 0; ok && j < npairs; ++j) {
-        if (j + 1 < npairs && !(ok = issue_qk(j + 1))) break;
-        if (!(ok = mbar_wait(smem_u32(&bar_pfull), j & 1, st, tmo, kWaitPFull))) break;
+        const int w = j & 1;
+        if (!(ok = mbar_wait(smem_u32(&bar_pfull[w]), (j >> 1) & 1, st, tmo, kWaitPFull))) break;
         const int s = j % C::kVSt;
         if (!(ok = mbar_wait(smem_u32(&bar_vfull[s]), (j / C::kVSt) & 1, st, tmo, kWaitVFull))) break;
         tc_fence_after();
         const int nb = min(2, cnt - 2 * j);
-        const uint32_t vb = sV0 + s * C::kKVBytes;
-        for (int kk = 0; kk < nb * 4; ++kk) {
-          const uint64_t bdesc = sw128_desc(vb + kk * 2048, C::kChunk, 1024);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (kPInTmem) {
-            umma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bdesc, idesc_pv, acc);
-          } else {
-            const uint32_t pa = sP + (kk >> 2) * C::kChunk + (kk & 3) * 32;
-            umma_ss(tmem + C::kColO, sw128_desc(pa, 16, 1024), bdesc, idesc_pv, acc);
+        const uint64_t vd = sw128_desc(sV0 + s * C::kKVBytes, C::kChunk, 1024);
+        const uint64_t pd = sw128_desc(sP0 + w * C::kPBytes, 16, 1024);
+        const uint32_t od = tmem + C::kColO + w * D;
+        const uint32_t acc0 = j >= 2 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          if (kk < nb * 4) {
+            const uint32_t poff = ((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4;
+            umma_ss(od, pd + poff, vd + kk * (2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
           }
         }
-        umma_commit(smem_u32(&bar_odone));
+        umma_commit(smem_u32(&bar_pfree[w]));
         umma_commit(smem_u32(&bar_vempty[s]));
       }
+      umma_commit(smem_u32(&bar_odone));
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x - 128;  // query row in the tile == TMEM lane
+  } else {
+    setmaxnreg_inc<C::kRegSm>();
+    // ------------------------------------------------ softmax warpgroups
+    const int w = (warp >> 2) - 1;                   // 0: even pairs, 1: odd pairs
+    const int row = threadIdx.x - 128 * (w + 1);     // query row in the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sbuf = tmem + lane_off + C::kColS + w * 128;
+    const uint32_t obuf = tmem + lane_off + C::kColO + w * D;
+    // Row `row` of this warpgroup's P tile (keys 0-63 in the first 16 KB
+    // chunk, keys 64-127 in the second), K-major with the 128-byte swizzle.
+    const uint32_t prow = sP0 + w * C::kPBytes + (row >> 3) * 1024 + (row & 7) * 128;
     const float sl2 = a.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     const int kb_last = a.Kb - 1;
     const int tail = a.N - kb_last * kBlockK;  // valid keys in the last key block (1..64)
+    const bool ragged = tail < 64 && s_last == kb_last;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < npairs; ++j) {
-      ok = mbar_wait(smem_u32(&bar_sfull[j & 1]), (j >> 1) & 1, st, tmo, kWaitSFull);
+    int t = 0;
+    for (int j = w; j < npairs; j += 2, ++t) {
+      ok = mbar_wait(smem_u32(&bar_sfull[w]), t & 1, st, tmo, kWaitSFull);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const int nb = min(2, cnt - 2 * j);
       float s[128];
-      const uint32_t sbuf = tmem + lane_off + C::kColS + (j & 1) * 128;
-      tmem_ld64(sbuf, s);
-      if (nb == 2) {
-        tmem_ld64(sbuf + 64, s + 64);
-      } else {
+      tmem_ld64_nowait(sbuf, s);
+      if (nb == 2) tmem_ld64_nowait(sbuf + 64, s + 64);
+      tmem_wait_ld();
+      reg_fence<128>(s);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_sfree[w]));  // S buffer may now receive S_{j+2}
+      if (nb != 2) {
 #pragma unroll
         for (int c = 64; c < 128; ++c) s[c] = -INFINITY;
       }
-      if (tail < 64) {
-        const bool last0 = s_idx[2 * j] == kb_last;
-        const bool last1 = nb == 2 && s_idx[2 * j + 1] == kb_last;
+      if (ragged && j == npairs - 1) {  // the last kept block is the ragged last key block
+        if (nb == 1) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (last0 && c >= tail) s[c] = -INFINITY;
-          if (last1 && c >= tail) s[64 + c] = -INFINITY;
+          for (int c = 0; c < 64; ++c) s[c] = c >= tail ? -INFINITY : s[c];
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[64 + c] = c >= tail ? -INFINITY : s[64 + c];
         }
       }
-      float mx[8];
+      float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = s[e];
-#pragma unroll
-      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 6; c < 126; c += 4) {
+        mx0 = fmax3(mx0, s[c], s[c + 1]);
+        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+      }
+      const float rmax = fmax3(mx0, mx1, fmaxf(s[126], s[127]));
       const float m_new = fmaxf(m_run, rmax * sl2);
       const bool need = m_new > m_run + 8.0f;  // always true for the first pair
       const float m_use = need ? m_new : m_run;
       const float alpha = ex2_approx(m_run - m_use);  // 0 for the first pair, 1 if no rescale
+      const uint64_t negm = f2_pack(-m_use, -m_use);
+      // Exponentials of column pairs: x = s * log2(e)/sqrt(d) - m as one f32x2
+      // FMA; the pairs selected by kPolyPattern on the FMA-pipe polynomial,
+      // the rest on MUFU.
       uint32_t pk[64];
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, -m_use));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -m_use));
-        ps[c & 3] += p0 + p1;
+        if (c >= 32 && nb != 2) break;
+        const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm);
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        uint64_t pp;
+        if ((kPolyPattern >> (c & 7)) & 1) {
+          pp = exp2_poly2(x0, x1);
+        } else {
+          pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[c & 1] = f2_add(acc[c & 1], pp);
+        float p0, p1;
+        f2_unpack(pp, p0, p1);
         pk[c] = pack_bf16(p0, p1);
       }
-      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      if (j > 0) {
-        // O and the P buffer are free once the previous P.V has completed.
-        ok = mbar_wait(smem_u32(&bar_odone), (j - 1) & 1, st, tmo, kWaitODone);
+      float a0, a1, a2, a3;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], a2, a3);
+      l_run = l_run * alpha + ((a0 + a1) + (a2 + a3));
+      // P buffer and O_w are free once this warpgroup's previous P.V is done.
+      if (t > 0) {
+        ok = mbar_wait(smem_u32(&bar_pfree[w]), (t - 1) & 1, st, tmo, kWaitPFree);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             float o[32];
-            const uint32_t oaddr = tmem + lane_off + C::kColO + cc * 32;
-            tmem_ld32(oaddr, o);
+            tmem_ld32(obuf + cc * 32, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(oaddr, reinterpret_cast<const uint32_t*>(o));
+            tmem_st32(obuf + cc * 32, reinterpret_cast<const uint32_t*>(o));
           }
+          tmem_wait_st();
         }
       }
-      if constexpr (kPInTmem) {
-        tmem_st32(tmem + lane_off + C::kColP, pk);
-        if (nb == 2) tmem_st32(tmem + lane_off + C::kColP + 32, pk + 32);
-      } else {
-        // Row `row` of the K-major, 128-byte-swizzled P tile (keys 0-63 in the
-        // first 16 KB chunk, keys 64-127 in the second).
-        const uint32_t rbase = sP + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && nb != 2) break;
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const uint32_t addr = rbase + h * C::kChunk + ((g ^ (row & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                         "r"(pk[h * 32 + g * 4]), "r"(pk[h * 32 + g * 4 + 1]),
-                         "r"(pk[h * 32 + g * 4 + 2]), "r"(pk[h * 32 + g * 4 + 3])
-                         : "memory");
-          }
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t addr = prow + h * C::kChunk + ((g ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(pk[h * 32 + g * 4]), "r"(pk[h * 32 + g * 4 + 1]),
+                       "r"(pk[h * 32 + g * 4 + 2]), "r"(pk[h * 32 + g * 4 + 3])
+                       : "memory");
         }
-        fence_proxy_async_smem();
       }
-      tmem_wait_st();
+      fence_proxy_async_smem();  // make P visible to the tensor core's async proxy
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_pfull));
+      mbar_arrive(smem_u32(&bar_pfull[w]));
       m_run = m_use;
     }
+    // ---------------------------------------------- epilogue: merge O_0, O_1
+    // Each warpgroup's (m, l) for its row go through shared memory (the P
+    // tiles, idle once every P.V has completed); then warpgroup w writes
+    // output columns [w D/2, (w+1) D/2) of its row.
     if (ok) {
-      ok = mbar_wait(smem_u32(&bar_odone), (npairs - 1) & 1, st, tmo, kWaitODone);
+      ok = mbar_wait(smem_u32(&bar_odone), 0, st, tmo, kWaitODone);
       ok = __all_sync(0xffffffffu, ok);
     }
+    float* xch = reinterpret_cast<float*>(dsmem + (sP0 - smem_u32(dsmem)));  // [2][128] m, [2][128] l
     if (ok) {
+      xch[w * 128 + row] = m_run;
+      xch[256 + w * 128 + row] = l_run;
+    } else if (lane == 0) {
+      s_fail = 1;
+    }
+    named_bar_sync(1, 256);
+    if (s_fail == 0) {
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      const bool has1 = npairs > 1;  // warpgroup 1 saw at least one pair
+      const float m0 = xch[row], m1 = xch[128 + row];
+      const float m = has1 ? fmaxf(m0, m1) : m0;
+      const float a0 = ex2_approx(m0 - m);
+      const float a1 = has1 ? ex2_approx(m1 - m) : 0.f;
+      const float inv = 1.f / (xch[256 + row] * a0 + (has1 ? xch[384 + row] * a1 : 0.f));
+      const float c0 = a0 * inv, c1 = a1 * inv;
       __nv_bfloat16* orow = out_blk + static_cast<size_t>(row) * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + C::kColO + cc * 32, o);
-        uint32_t w[16];
+      for (int cc = w * (D / 64); cc < (w + 1) * (D / 64); ++cc) {
+        float o0[32], o1[32];
+        tmem_ld32(tmem + lane_off + C::kColO + cc * 32, o0);
+        if (has1) {
+          tmem_ld32(tmem + lane_off + C::kColO + D + cc * 32, o1);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+          for (int e = 0; e < 32; ++e) o1[e] = 0.f;
+        }
+        uint32_t wv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          wv[e] = pack_bf16(fmaf(o0[2 * e], c0, o1[2 * e] * c1), fmaf(o0[2 * e + 1], c0, o1[2 * e + 1] * c1));
         if (row < rows_valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
         }
       }
     }
@@ -368,7 +444,7 @@ __global__ void __launch_bounds__(256, 1)
     for (int s = 0; s < nst; ++s) {
       if (issued[s] == 0) continue;
       const uint32_t bar = smem_u32(warp == 0 ? &bar_kfull[s] : &bar_vfull[s]);
-      uint64_t t0 = globaltimer_ns();
+      const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(bar, (issued[s] - 1) & 1)) {
         if (globaltimer_ns() - t0 > tmo) {
           atomicCAS(&st->code, 0u, kDevTimeout);
@@ -377,7 +453,7 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     if (warp == 0) {
-      uint64_t t0 = globaltimer_ns();
+      const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(smem_u32(&bar_q), 0)) {
         if (globaltimer_ns() - t0 > tmo) {
           atomicCAS(&st->code, 0u, kDevTimeout);
@@ -386,11 +462,12 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   }
-  if (warp == 1) {
-    if (lane == 0) {
-      umma_commit(smem_u32(&bar_final));
-      uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(&bar_final), 0)) {
+  if (warp == 1 || warp == 3) {
+    if (lane == 0 && mma_issued) {
+      // Each issuer committed a final barrier after its last MMA; wait for it (bounded).
+      const uint32_t fin = smem_u32(warp == 1 ? &bar_qkdone : &bar_odone);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(fin, 0)) {
         if (globaltimer_ns() - t0 > tmo) {
           atomicCAS(&st->code, 0u, kDevTimeout);
           break;
@@ -444,23 +521,19 @@ bool make_map(CUtensorMap* m, const void* ptr, int BH, int N, int D, int box_row
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kPInTmem>
+template <int D>
 cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttnArgs& args, int BH, cudaStream_t st) {
-  using C = Cfg<D, kPInTmem>;
-  auto kern = bsa_fwd_kernel<D, kPInTmem>;
+  using C = Cfg<D>;
+  auto kern = bsa_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(args.Qb);
-  kern<<<grid, 256, C::kSmem, st>>>(mq, mk, mv, args);
+  kern<<<grid, C::kThreads, C::kSmem, st>>>(mq, mk, mv, args);
   return cudaGetLastError();
 }
 
 }  // namespace
-
-#ifndef BSA_P_IN_TMEM
-#define BSA_P_IN_TMEM 1
-#endif
 
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, int BH, int N,
                              int d, const int16_t* idx, const int32_t* cnt, DeviceStatus* status,
@@ -481,8 +554,8 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
   args.Qb = (N + kBlockQ - 1) / kBlockQ;
   args.Kb = (N + kBlockK - 1) / kBlockK;
   args.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
-  if (d == 128) return launch_typed<128, BSA_P_IN_TMEM != 0>(mq, mk, mv, args, BH, st);
-  return launch_typed<64, BSA_P_IN_TMEM != 0>(mq, mk, mv, args, BH, st);
+  if (d == 128) return launch_typed<128>(mq, mk, mv, args, BH, st);
+  return launch_typed<64>(mq, mk, mv, args, BH, st);
 }
 
 }  // namespace bsa

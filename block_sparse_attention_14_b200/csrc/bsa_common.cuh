@@ -59,6 +59,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended in hardware for up to
+// `hint_ns` while the phase is still pending (no busy spinning).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity of `bar` has completed.  The
 // wait is bounded: it gives up when `timeout_ns` have passed or when another
 // CTA has already recorded a failure in `st`; on giving up it records the
@@ -67,19 +82,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceS
                                           uint64_t timeout_ns, uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*reinterpret_cast<volatile uint32_t*>(&st->code) != 0) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
-        if (atomicCAS(&st->code, 0u, kDevTimeout) == 0u) {
-          st->where = where;
-          st->block = blockIdx.x;
-        }
-        return false;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*reinterpret_cast<volatile uint32_t*>(&st->code) != 0) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      if (atomicCAS(&st->code, 0u, kDevTimeout) == 0u) {
+        st->where = where;
+        st->block = blockIdx.x;
       }
+      return false;
     }
   }
+}
+
+// Register budget of the calling warpgroup (all four warps must execute it).
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Named barrier over `count` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---------------------------------------------------------------------- TMA
@@ -217,6 +245,42 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
       : "memory");
 }
 
+// Two 32-column loads without waiting; the caller waits with tmem_wait_ld()
+// and then passes the registers through reg_fence() before using them.
+__device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, "
+      "%42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, "
+      "%60, %61, %62, %63}, [%65];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr), "r"(taddr + 32u)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Orders later uses of v after a preceding tmem_wait_ld() (volatile asm
+// statements keep their relative order, and every use now depends on it).
+template <int N>
+__device__ __forceinline__ void reg_fence(float* v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 // Store 32 lanes x 32 columns of 32-bit words (thread t writes its lane).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -239,6 +303,71 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Software 2^x on the FMA and integer pipes, so that part of the softmax
+// exponentials leave the MUFU unit.  Cody-Waite style split x = n + f with
+// n = round(x) (the 1.5 * 2^23 shifter leaves n in the low mantissa bits of t)
+// and f in [-1/2, 1/2]; 2^f is a degree-4 polynomial whose coefficients are a
+// Remez minimax fit of the relative error (exp2_poly_fit.py, max relative
+// error 2.7e-6); 2^n is added into the exponent field.  Inputs below -126
+// (including -inf) return 2^-126 * p(0) ~ 1.2e-38 instead of 0, which is
+// negligible next to the row maximum's weight of 1.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(9.570102207e-03f, f, 5.591785908e-02f);
+  p = fmaf(p, f, 2.402474433e-01f);
+  p = fmaf(p, f, 6.931217909e-01f);
+  p = fmaf(p, f, 9.999992847e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic: two lanes per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_poly on a packed pair: clamp, shifter and Horner steps run as f32x2.
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t nmag = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t n = f2_add(t, nmag);
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);  // x - n, exact
+  uint64_t p = f2_fma(f2_pack(9.570102207e-03f, 9.570102207e-03f), f,
+                      f2_pack(5.591785908e-02f, 5.591785908e-02f));
+  p = f2_fma(p, f, f2_pack(2.402474433e-01f, 2.402474433e-01f));
+  p = f2_fma(p, f, f2_pack(6.931217909e-01f, 6.931217909e-01f));
+  p = f2_fma(p, f, f2_pack(9.999992847e-01f, 9.999992847e-01f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
