@@ -91,6 +91,12 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 
+uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+
+void set_last_error(const char* msg) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+}
+
 size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base) {
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t Qb = (static_cast<size_t>(N) + kBlockQ - 1) / kBlockQ;

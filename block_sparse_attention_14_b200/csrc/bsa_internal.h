@@ -21,6 +21,12 @@ struct Workspace {
 
 size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base);
 
+// Current limit of the kernels' bounded waits (bsa_set_wait_timeout_ns).
+uint64_t wait_timeout_ns();
+
+// Records the message returned by bsa_last_error_message() on this thread.
+void set_last_error(const char* msg);
+
 // (a1, a2) mean-pool q over 128-row blocks and k over 64-row blocks.
 cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, float* qbar,
                         float* kbar, cudaStream_t st);

@@ -1,0 +1,97 @@
+// sparse_attn_topk_noalloc: the fused selection + attention call for callers
+// that cannot allocate device memory.  Its scratch (pooled means, kept-block
+// lists, status word) lives in a file-scope __device__ array instead of a
+// caller-provided workspace; the caller still passes q, k, v, out and mask.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "bsa.h"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+// 32 MiB, held by every GPU that loads the library until the process exits.
+constexpr size_t kStaticScratchBytes = 32ull << 20;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of g_static_scratch.  In host code the
+// symbol's name is only a host-side handle, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+bsa_status reject(bsa_status s, const char* msg) {
+  set_last_error(msg);
+  return s;
+}
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
+                                               bsa_shape s, float topk, int is_causal, void* out,
+                                               uint8_t* mask_out, void* stream) {
+  set_last_error("");
+  if (s.B < 1 || s.H < 1 || s.N < 1 || (s.d != 64 && s.d != 128) || s.N > kBlockK * kMaxKb ||
+      static_cast<int64_t>(s.B) * s.H > 65535)
+    return reject(BSA_ERR_INVALID_ARG, "bad shape: need B, H, N >= 1, d in {64, 128}, N <= 131072, B*H <= 65535");
+  if (is_causal != 0) return reject(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
+  const void* ptrs[4] = {q, k, v, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0)
+      return reject(BSA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
+  if (!(topk > 0.f) || !(topk <= 1.f)) return reject(BSA_ERR_INVALID_ARG, "topk must lie in (0, 1]");
+  const size_t need = workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr);
+  if (need > kStaticScratchBytes) {
+    char msg[200];
+    snprintf(msg, sizeof(msg),
+             "this shape needs %zu bytes of scratch; the static scratch of the no-allocation call "
+             "holds %zu bytes (use sparse_attn_topk with a caller workspace)",
+             need, kStaticScratchBytes);
+    return reject(BSA_ERR_INVALID_ARG, msg);
+  }
+  void* base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess) return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
+  Workspace w;
+  workspace_layout(s.B, s.H, s.N, s.d, &w, base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  const int Kb = (s.N + kBlockK - 1) / kBlockK;
+  long long kk = static_cast<long long>(ceil(static_cast<double>(topk) * static_cast<double>(Kb)));
+  kk = kk < 1 ? 1 : (kk > Kb ? Kb : kk);
+  // The status word must start at zero; everything else is overwritten.
+  if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
+      (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
+      (e = launch_select(w.qbar, w.kbar, BH, s.N, s.d, static_cast<int>(kk), mask_out, w.idx, w.cnt,
+                         st)) != cudaSuccess)
+    return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
+  const char* why = nullptr;
+  e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status, wait_timeout_ns(), st, &why);
+  if (e != cudaSuccess) return reject(BSA_ERR_CUDA, why ? why : cudaGetErrorString(e));
+  return BSA_OK;
+}

@@ -123,6 +123,26 @@ bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, void* ws,
 bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, bsa_shape s,
                                    void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* No-allocation variant of sparse_attn_topk (same arguments minus the
+ * workspace; same kernels, same results).  The pages have no counterpart: this
+ * call exists for callers that cannot allocate device memory, such as a
+ * serving engine that reserves all free device memory for its own pool at
+ * start-up (so no memory is left for a workspace), or a caller on a
+ * latency-critical path that must not trigger the device-wide synchronisation
+ * of cudaFree.  Its scratch is a file-scope device array of 32 MiB, held on
+ * every GPU that loads the library until the process exits; shapes whose
+ * workspace (bsa_workspace_bytes) exceeds 32 MiB are rejected with
+ * BSA_ERR_INVALID_ARG before anything is launched.  The first call on a device
+ * looks up that device's copy of the array with cudaGetSymbolAddress (with the
+ * device current), so make the first call on each device before any stream
+ * capture.  Every call on a device shares the one array: calls that may
+ * overlap on the GPU (different streams, other threads) race and corrupt each
+ * other's results, so order them on one stream.  The call allocates nothing.
+ * mask_out is optional (NULL: not written). */
+bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v, bsa_shape s,
+                                    float topk, int is_causal, void* out, uint8_t* mask_out,
+                                    void* stream);
+
 /* Synchronises `stream`, then reports what the kernels of the last call that
  * used `ws` recorded: BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out), or
  * BSA_ERR_CUDA if the stream holds an error. */
