@@ -156,13 +156,20 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of a per-rank scalar (a step time) over all ranks."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(dense_flops_per_rank: float, step_s_max: float, world: int) -> float:
+    """Weak scaling: every rank runs one call; throughput of all ranks over the slowest one."""
+    return world * dense_flops_per_rank / step_s_max / 1e12
 
 
 def barrier(world: int):
@@ -366,7 +373,7 @@ def run_b200(args, world, rank, local):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": world * dense_flops / step_max / 1e12, "unit": UNIT,
+            "metric": METRIC, "value": whole_job_value(dense_flops, step_max, world), "unit": UNIT,
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": step_max * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(wl, args.topk, H),

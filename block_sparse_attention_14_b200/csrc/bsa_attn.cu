@@ -43,7 +43,9 @@ namespace {
 #ifndef BSA_POLY_PATTERN
 #define BSA_POLY_PATTERN 0x88
 #endif
-constexpr unsigned kPolyPattern = BSA_POLY_PATTERN;
+#ifndef BSA_POLY_PATTERN_D64
+#define BSA_POLY_PATTERN_D64 0x88
+#endif
 
 enum WaitSite : uint32_t {
   kWaitQ = 1,
@@ -86,6 +88,7 @@ struct Cfg {
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr unsigned kPolyPattern = (D == 64) ? BSA_POLY_PATTERN_D64 : BSA_POLY_PATTERN;
   static constexpr uint32_t kRegCtl = 56;   // registers per thread, control warpgroup
   static constexpr uint32_t kRegSm = 224;   // registers per thread, softmax warpgroups
   static_assert(kSmem + 512 <= 227 * 1024, "shared memory budget (dynamic + static)");
@@ -295,10 +298,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const int nb = min(2, cnt - 2 * j);
       float s[128];
-      tmem_ld64_nowait(sbuf, s);
-      if (nb == 2) tmem_ld64_nowait(sbuf + 64, s + 64);
-      tmem_wait_ld();
-      reg_fence<128>(s);
+      tmem_ld128(sbuf, s);  // for an odd last block the upper 64 columns are stale and overwritten below
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_sfree[w]));  // S buffer may now receive S_{j+2}
       if (nb != 2) {
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(384, 1)
       const float alpha = ex2_approx(m_run - m_use);  // 0 for the first pair, 1 if no rescale
       const uint64_t negm = f2_pack(-m_use, -m_use);
       // Exponentials of column pairs: x = s * log2(e)/sqrt(d) - m as one f32x2
-      // FMA; the pairs selected by kPolyPattern on the FMA-pipe polynomial,
+      // FMA; the pairs selected by C::kPolyPattern on the FMA-pipe polynomial,
       // the rest on MUFU.
       uint32_t pk[64];
       uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(384, 1)
         float x0, x1;
         f2_unpack(x, x0, x1);
         uint64_t pp;
-        if ((kPolyPattern >> (c & 7)) & 1) {
+        if ((C::kPolyPattern >> (c & 7)) & 1) {
           pp = exp2_poly2(x0, x1);
         } else {
           pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
