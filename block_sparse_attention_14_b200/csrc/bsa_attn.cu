@@ -438,7 +438,10 @@ __global__ void __launch_bounds__(384, 1)
   // ---------------------------------------------------------------- teardown
   // Every role has left its loop (finished, or gave up after a bounded wait).
   // Drain what may still be in flight before the TMEM is released and the CTA
-  // exits: outstanding TMA loads (producers) and tensor-core ops (issuer).
+  // exits: outstanding TMA loads (producers) and tensor-core ops (issuers).
+  // Those always finish within microseconds, so the drain waits up to at
+  // least 100 ms even when the caller set a shorter wait limit.
+  const uint64_t drain = tmo > 100000000ull ? tmo : 100000000ull;
   __syncthreads();
   if ((warp == 0 || warp == 2) && lane == 0) {
     const int nst = (warp == 0) ? C::kKSt : C::kVSt;
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t bar = smem_u32(warp == 0 ? &bar_kfull[s] : &bar_vfull[s]);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(bar, (issued[s] - 1) & 1)) {
-        if (globaltimer_ns() - t0 > tmo) {
+        if (globaltimer_ns() - t0 > drain) {
           atomicCAS(&st->code, 0u, kDevTimeout);
           break;
         }
@@ -456,7 +459,7 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 0) {
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(smem_u32(&bar_q), 0)) {
-        if (globaltimer_ns() - t0 > tmo) {
+        if (globaltimer_ns() - t0 > drain) {
           atomicCAS(&st->code, 0u, kDevTimeout);
           break;
         }
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t fin = smem_u32(warp == 1 ? &bar_qkdone : &bar_odone);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(fin, 0)) {
-        if (globaltimer_ns() - t0 > tmo) {
+        if (globaltimer_ns() - t0 > drain) {
           atomicCAS(&st->code, 0u, kDevTimeout);
           break;
         }
