@@ -112,11 +112,83 @@ def topk_mask(P: np.ndarray, k: int) -> np.ndarray:
     return mask.reshape(P.shape)
 
 
-def select(q, k, topk: float):
+def cdf_mask(P: np.ndarray, threshold: float) -> np.ndarray:
+    """cdfthreshd selection ("SpargeAttention Documentation", the --mode
+    cdfthreshd flag of the inference scripts; the pages print no formula).
+
+    Reading: order each row by P descending (equal scores: lower index first)
+    and keep the shortest prefix whose cumulative mass reaches the threshold,
+    at least one block.  If rounding leaves the total mass below the threshold,
+    the whole row is kept.  threshold is taken as its float32 value.
+    """
+    tau = float(np.float32(threshold))
+    Kb = P.shape[-1]
+    rows = P.reshape(-1, Kb)
+    mask = np.zeros(rows.shape, dtype=np.uint8)
+    j = np.arange(Kb)
+    for r in range(rows.shape[0]):
+        order = np.lexsort((j, -rows[r]))
+        cum = np.cumsum(rows[r][order])
+        m = int(np.searchsorted(cum, tau, side="left"))  # first prefix whose sum >= tau
+        mask[r, order[:min(m, Kb - 1) + 1]] = 1
+    return mask.reshape(P.shape)
+
+
+def select_cdf(q, k, threshold: float):
+    """Mean-pool, score and cdfthreshd-select.  Returns (mask uint8, P float64)."""
+    _, P = select(q, k, 1.0)
+    return cdf_mask(P, threshold), P
+
+
+def cdf_exempt_rows(P: np.ndarray, threshold: float, tol: float = 1e-4, tie_rel: float = 1e-6) -> np.ndarray:
+    """Rows whose cdfthreshd decision is not determined at the precision of the
+    inputs: the threshold lies within `tol` of a cumulative sum next to the cut,
+    or the scores around the cut tie to within `tie_rel`."""
+    tau = float(np.float32(threshold))
+    Kb = P.shape[-1]
+    rows = P.reshape(-1, Kb)
+    ex = np.zeros(rows.shape[0], dtype=bool)
+    j = np.arange(Kb)
+    for r in range(rows.shape[0]):
+        order = np.lexsort((j, -rows[r]))
+        ps = rows[r][order]
+        cum = np.cumsum(ps)
+        m = min(int(np.searchsorted(cum, tau, side="left")), Kb - 1)
+        near = abs(cum[m] - tau) < tol or (m > 0 and abs(cum[m - 1] - tau) < tol)
+        tie = m + 1 < Kb and (ps[m] - ps[m + 1]) < tie_rel * ps[m]
+        ex[r] = near or tie
+    return ex.reshape(P.shape[:-1])
+
+
+def causal_block_limit(i: int, Kb: int) -> int:
+    """Number of key blocks that query block i may use under causal attention.
+
+    Reading (is_causal is exposed by the recommended API on "SpargeAttention
+    Documentation" but not described): key block j holds keys 64 j .. 64 j + 63
+    and query block i rows 128 i .. 128 i + 127, so a key of block j precedes
+    some row of block i exactly when j <= 2 i + 1.
+    """
+    return min(2 * i + 2, Kb)
+
+
+def causal_topk_mask(P: np.ndarray, topk: float) -> np.ndarray:
+    """Top-k among each row's causally eligible key blocks: row i keeps
+    keep_count(topk, E_i) of its E_i = causal_block_limit(i, Kb) eligible blocks,
+    equal scores to the lower index; ineligible blocks are never kept."""
+    B, H, Qb, Kb = P.shape
+    mask = np.zeros(P.shape, dtype=np.uint8)
+    for i in range(Qb):
+        E = causal_block_limit(i, Kb)
+        mask[:, :, i, :E] = topk_mask(P[:, :, i:i + 1, :E], keep_count(topk, E))[:, :, 0]
+    return mask
+
+
+def select(q, k, topk: float, causal: bool = False):
     """Mean-pool, score and top-k select.  Returns (mask uint8, P float64).
 
     q and k may be bf16 torch tensors; they are upcast one (b, h) slice at a
-    time so that full-size inputs fit in host memory.
+    time so that full-size inputs fit in host memory.  With causal=True the
+    top-k runs over each row's eligible key blocks (causal_topk_mask).
     """
     B, H, N, d = q.shape
     Qb, Kb = block_counts(N)
@@ -127,6 +199,8 @@ def select(q, k, topk: float):
             qbar[b, h] = pool_mean(to_f64(q[b, h])[None, None], BLOCK_Q)[0, 0]
             kbar[b, h] = pool_mean(to_f64(k[b, h])[None, None], BLOCK_K)[0, 0]
     P = block_scores(qbar, kbar)
+    if causal:
+        return causal_topk_mask(P, topk), P
     return topk_mask(P, keep_count(topk, Kb)), P
 
 
@@ -137,14 +211,16 @@ def kept_key_columns(mask_row: np.ndarray, N: int) -> np.ndarray:
 
 
 def attention_rows(qh: np.ndarray, kh: np.ndarray, vh: np.ndarray, mask_row: np.ndarray,
-                   i: int) -> np.ndarray:
+                   i: int, causal: bool = False) -> np.ndarray:
     """Output rows [128 i, min(128 i + 128, N)) of one head -> [rows, d] float64.
 
     qh, kh, vh are that head's [N, d] float64 arrays and mask_row its Kb mask
     entries for query block i.  Softmax over the union of the kept key blocks
     (nonzero entries), scale 1/sqrt(d) as in scaled-dot-product attention,
     taken in two passes (row max, then exponentials and their sum).  Reading: a
-    query block with no kept key block produces zeros.
+    query block with no kept key block produces zeros.  With causal=True only
+    keys at or before the row's own position count, and a row left with no
+    such key produces zeros too.
     """
     N, d = qh.shape
     lo, hi = i * BLOCK_Q, min((i + 1) * BLOCK_Q, N)
@@ -152,13 +228,20 @@ def attention_rows(qh: np.ndarray, kh: np.ndarray, vh: np.ndarray, mask_row: np.
     if cols.size == 0:
         return np.zeros((hi - lo, d), dtype=np.float64)
     S = qh[lo:hi] @ kh[cols].T / math.sqrt(d)
+    if causal:
+        S = np.where(cols[None, :] <= np.arange(lo, hi)[:, None], S, -np.inf)
     m = S.max(axis=1, keepdims=True)
-    E = np.exp(S - m)
-    return (E @ vh[cols]) / E.sum(axis=1, keepdims=True)
+    out = np.zeros((hi - lo, d), dtype=np.float64)
+    live = np.isfinite(m[:, 0])
+    if live.any():
+        E = np.exp(S[live] - m[live])
+        out[live] = (E @ vh[cols]) / E.sum(axis=1, keepdims=True)
+    return out
 
 
-def block_sparse_attention(q, k, v, mask) -> np.ndarray:
-    """Full output [B, H, N, d] float64 of attention restricted to the kept tiles."""
+def block_sparse_attention(q, k, v, mask, causal: bool = False) -> np.ndarray:
+    """Full output [B, H, N, d] float64 of attention restricted to the kept tiles
+    (and, with causal=True, to keys at or before each row)."""
     mask = np.asarray(mask)
     B, H, N, d = q.shape
     Qb, Kb = block_counts(N)
@@ -168,7 +251,8 @@ def block_sparse_attention(q, k, v, mask) -> np.ndarray:
         for h in range(H):
             qh, kh, vh = to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h])
             for i in range(Qb):
-                out[b, h, i * BLOCK_Q:min((i + 1) * BLOCK_Q, N)] = attention_rows(qh, kh, vh, mask[b, h, i], i)
+                out[b, h, i * BLOCK_Q:min((i + 1) * BLOCK_Q, N)] = attention_rows(qh, kh, vh, mask[b, h, i], i,
+                                                                                  causal)
     return out
 
 

@@ -330,9 +330,126 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     good_rows = mod.attention_rows
 
-    def rows_transposed_mask(qh, kh, vh, mask_row, i):  # uses the complement of the mask
-        return good_rows(qh, kh, vh, (np.asarray(mask_row) == 0).astype(np.uint8), i)
+    def rows_transposed_mask(qh, kh, vh, mask_row, i, causal=False):  # uses the complement of the mask
+        return good_rows(qh, kh, vh, (np.asarray(mask_row) == 0).astype(np.uint8), i, causal)
 
     monkeypatch.setattr(mod, "attention_rows", rows_transposed_mask)
     assert fails(lambda: test_block_mask_equals_sdpa_with_expanded_token_mask(300))
     monkeypatch.setattr(mod, "attention_rows", good_rows)
+
+    def rows_off_by_one_causal(qh, kh, vh, mask_row, i, causal=False):  # excludes the diagonal key
+        if not causal:
+            return good_rows(qh, kh, vh, mask_row, i)
+        N, d = qh.shape
+        lo, hi = i * 128, min((i + 1) * 128, N)
+        cols = mod.kept_key_columns(mask_row, N)
+        S = qh[lo:hi] @ kh[cols].T / math.sqrt(d)
+        S = np.where(cols[None, :] < np.arange(lo, hi)[:, None], S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        out = np.zeros((hi - lo, d))
+        live = np.isfinite(m[:, 0])
+        E = np.exp(S[live] - m[live])
+        out[live] = (E @ vh[cols]) / E.sum(axis=1, keepdims=True)
+        return out
+
+    monkeypatch.setattr(mod, "attention_rows", rows_off_by_one_causal)
+    assert fails(lambda: test_causal_all_ones_equals_library_causal_sdpa(300))
+    monkeypatch.setattr(mod, "attention_rows", good_rows)
+
+
+# ---------------------------------------------------------------- cdfthreshd
+def _brute_cdf(row, tau):
+    """Smallest subset reaching mass tau; among those the largest mass, then the
+    lexicographically smallest index set."""
+    n = len(row)
+    for size in range(1, n + 1):
+        best, best_set = None, None
+        for sub in itertools.combinations(range(n), size):
+            s = sum(row[j] for j in sub)
+            if s >= tau and (best is None or s > best):
+                best, best_set = s, sub
+        if best_set is not None:
+            return best_set
+    return tuple(range(n))
+
+
+def test_cdf_mask_matches_brute_force():
+    rng = _rng(21)
+    for trial in range(60):
+        Kb = int(rng.integers(1, 10))
+        row = rng.random(Kb) ** 3
+        row = row / row.sum()
+        tau = float(np.float32(rng.uniform(0.05, 0.999)))
+        got = tuple(np.flatnonzero(O.cdf_mask(row[None, None, None], tau)[0, 0, 0]))
+        assert got == _brute_cdf(list(row), tau), (row, tau)
+
+
+def test_cdf_mask_closed_forms():
+    # Values exactly representable in float32, so the float32 threshold equals its
+    # decimal value.
+    row = np.array([0.125, 0.375, 0.25, 0.25])[None, None, None]
+    assert list(np.flatnonzero(O.cdf_mask(row, 0.375)[0, 0, 0])) == [1]        # 0.375 reaches 0.375
+    assert list(np.flatnonzero(O.cdf_mask(row, 0.5)[0, 0, 0])) == [1, 2]       # 0.625, tie -> lower index
+    assert list(np.flatnonzero(O.cdf_mask(row, 0.625)[0, 0, 0])) == [1, 2]
+    assert list(np.flatnonzero(O.cdf_mask(row, 0.75)[0, 0, 0])) == [1, 2, 3]   # 0.875
+    assert O.cdf_mask(row, 1.0)[0, 0, 0].sum() == 4
+    assert O.cdf_mask(row, 1e-6)[0, 0, 0].sum() == 1                           # at least one
+    # the threshold is read as float32: 0.4f > 0.4, so 0.4 alone no longer reaches it
+    row2 = np.array([0.1, 0.4, 0.2, 0.3])[None, None, None]
+    assert list(np.flatnonzero(O.cdf_mask(row2, 0.4)[0, 0, 0])) == [1, 3]
+
+
+def test_cdf_exempt_rows_flags_boundaries():
+    P = np.array([[[[0.5, 0.3, 0.2]], [[0.5, 0.25, 0.25 * (1 - 1e-9)]]]])
+    assert O.cdf_exempt_rows(P, 0.8)[0, 0, 0]       # 0.5 + 0.3 sits on the threshold
+    assert O.cdf_exempt_rows(P, 0.7)[0, 1, 0]       # kept and first dropped score tie
+    assert not O.cdf_exempt_rows(P, 0.6)[0, 0, 0]
+
+
+# -------------------------------------------------------------------- causal
+def test_causal_block_limit_hand_worked():
+    # query block i covers rows 128i..128i+127, so key blocks 0..2i+1 hold earlier keys
+    assert [O.causal_block_limit(i, 100) for i in range(4)] == [2, 4, 6, 8]
+    assert O.causal_block_limit(3, 5) == 5
+
+
+@pytest.mark.parametrize("N", [256, 300, 129, 1])
+def test_causal_all_ones_equals_library_causal_sdpa(N):
+    rng = _rng(31)
+    q, k, v = (rng.normal(size=(1, 2, N, 32)) for _ in range(3))
+    Qb, Kb = O.block_counts(N)
+    ones = np.ones((1, 2, Qb, Kb), dtype=np.uint8)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=True).numpy()
+    np.testing.assert_allclose(O.block_sparse_attention(q, k, v, ones, causal=True), want, rtol=0, atol=1e-12)
+
+
+def test_causal_block_mask_equals_sdpa_with_combined_mask():
+    rng = _rng(32)
+    N = 400
+    q, k, v = (rng.normal(size=(1, 3, N, 16)) * 2 for _ in range(3))
+    Qb, Kb = O.block_counts(N)
+    mask = (rng.random((1, 3, Qb, Kb)) < 0.5).astype(np.uint8)
+    mask[0, 0, 1] = 0
+    mask[0, 0, 1, 3] = 1          # only the second diagonal block: rows 128..191 see nothing
+    got = O.block_sparse_attention(q, k, v, mask, causal=True)
+    tok = _expand(mask, N) & np.tril(np.ones((N, N), dtype=bool))[None, None]
+    live = tok.any(-1)
+    want = _sdpa(q, k, v, attn_mask=tok)
+    np.testing.assert_allclose(got[live], want[live], rtol=0, atol=1e-12)
+    assert np.all(got[~live] == 0.0) and (~live).sum() >= 64
+
+
+def test_causal_topk_matches_brute_force_over_eligible_blocks():
+    rng = _rng(33)
+    for trial in range(20):
+        Qb = 3
+        Kb = int(rng.integers(2, 7))
+        P = rng.random((1, 1, Qb, Kb))
+        topk = float(rng.uniform(0.05, 1.0))
+        m = O.causal_topk_mask(P, topk)
+        for i in range(Qb):
+            E = O.causal_block_limit(i, Kb)
+            kk = O.keep_count(topk, E)
+            assert m[0, 0, i, E:].sum() == 0
+            assert tuple(np.flatnonzero(m[0, 0, i])) == _brute_topk(list(P[0, 0, i, :E]), kk)
