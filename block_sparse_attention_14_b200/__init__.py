@@ -30,7 +30,7 @@ import torch
 
 __all__ = [
     "BsaError", "sparse_attn_topk", "block_sparse_attn_fwd", "sparse_attn_select",
-    "sparse_attn_block_scores", "workspace_bytes", "make_workspace", "last_device_status",
+    "sparse_attn_block_scores", "sparse_attn_select_cdf", "sparse_attn_cdf", "workspace_bytes", "make_workspace", "last_device_status",
     "set_wait_timeout_ns", "block_sparse_attn_plan", "block_sparse_attn_apply", "block_counts", "keep_count", "library_path", "lib",
 ]
 
@@ -77,15 +77,19 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_block_scores.restype = i32
         L.sparse_attn_block_scores.argtypes = [vp, vp, Shape, vp, vp, sz, vp]
         L.sparse_attn_select.restype = i32
-        L.sparse_attn_select.argtypes = [vp, vp, Shape, f32, vp, vp, sz, vp]
+        L.sparse_attn_select.argtypes = [vp, vp, Shape, f32, i32, vp, vp, sz, vp]
         L.block_sparse_attn_fwd.restype = i32
         L.block_sparse_attn_fwd.argtypes = [vp, vp, vp, Shape, vp, i32, vp, vp, sz, vp]
         L.sparse_attn_topk.restype = i32
         L.sparse_attn_topk.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp, sz, vp]
+        L.sparse_attn_select_cdf.restype = i32
+        L.sparse_attn_select_cdf.argtypes = [vp, vp, Shape, f32, vp, vp, sz, vp]
+        L.sparse_attn_cdf.restype = i32
+        L.sparse_attn_cdf.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp, sz, vp]
         L.block_sparse_attn_plan.restype = i32
-        L.block_sparse_attn_plan.argtypes = [vp, Shape, vp, sz, vp]
+        L.block_sparse_attn_plan.argtypes = [vp, Shape, i32, vp, sz, vp]
         L.block_sparse_attn_apply.restype = i32
-        L.block_sparse_attn_apply.argtypes = [vp, vp, vp, Shape, vp, vp, sz, vp]
+        L.block_sparse_attn_apply.argtypes = [vp, vp, vp, Shape, i32, vp, vp, sz, vp]
         L.bsa_last_device_status.restype = i32
         L.bsa_last_device_status.argtypes = [vp, vp]
         L.bsa_set_wait_timeout_ns.restype = None
@@ -202,8 +206,10 @@ def block_sparse_attn_fwd(q, k, v, mask_id=None, is_causal: bool = False, *, out
     return out
 
 
-def sparse_attn_select(q, k, topk: float, *, mask_out=None, workspace=None) -> torch.Tensor:
-    """Selection mask alone: uint8 [B, H, ceil(N/128), ceil(N/64)]."""
+def sparse_attn_select(q, k, topk: float, is_causal: bool = False, *, mask_out=None,
+                       workspace=None) -> torch.Tensor:
+    """Selection mask alone: uint8 [B, H, ceil(N/128), ceil(N/64)].  With is_causal,
+    row i chooses among its key blocks 0 .. 2i+1 only."""
     _qkv(q, k)
     B, H, N, _ = q.shape
     if mask_out is None:
@@ -211,8 +217,37 @@ def sparse_attn_select(q, k, topk: float, *, mask_out=None, workspace=None) -> t
     mask_out = _mask_arg(mask_out, q)
     ws, wp, wn = _ws(q, workspace)
     _check(lib().sparse_attn_select(q.data_ptr(), k.data_ptr(), _shape_of(q), float(topk),
-                                    mask_out.data_ptr(), wp, wn, _stream(q)))
+                                    int(bool(is_causal)), mask_out.data_ptr(), wp, wn, _stream(q)))
     return mask_out
+
+
+def sparse_attn_select_cdf(q, k, threshold: float, *, mask_out=None, workspace=None) -> torch.Tensor:
+    """cdfthreshd selection mask: per row, the shortest score-ordered prefix of key
+    blocks whose block-score mass reaches `threshold` (uint8 [B, H, Qb, Kb])."""
+    _qkv(q, k)
+    B, H, N, _ = q.shape
+    if mask_out is None:
+        mask_out = torch.empty(B, H, *block_counts(N), dtype=torch.uint8, device=q.device)
+    mask_out = _mask_arg(mask_out, q)
+    ws, wp, wn = _ws(q, workspace)
+    _check(lib().sparse_attn_select_cdf(q.data_ptr(), k.data_ptr(), _shape_of(q), float(threshold),
+                                        mask_out.data_ptr(), wp, wn, _stream(q)))
+    return mask_out
+
+
+def sparse_attn_cdf(q, k, v, threshold: float = 0.9, is_causal: bool = False, *, out=None,
+                    return_mask: bool = False, workspace=None):
+    """cdfthreshd selection followed by block-sparse attention."""
+    _qkv(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    _qkv(q, out)
+    B, H, N, _ = q.shape
+    mask = torch.empty(B, H, *block_counts(N), dtype=torch.uint8, device=q.device) if return_mask else None
+    ws, wp, wn = _ws(q, workspace)
+    _check(lib().sparse_attn_cdf(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q), float(threshold),
+                                 int(bool(is_causal)), out.data_ptr(),
+                                 mask.data_ptr() if mask is not None else None, wp, wn, _stream(q)))
+    return (out, mask) if return_mask else out
 
 
 def sparse_attn_block_scores(q, k, *, out=None, workspace=None) -> torch.Tensor:
@@ -229,25 +264,25 @@ def sparse_attn_block_scores(q, k, *, out=None, workspace=None) -> torch.Tensor:
     return out
 
 
-def block_sparse_attn_plan(q, mask_id=None, *, workspace=None) -> torch.Tensor:
+def block_sparse_attn_plan(q, mask_id=None, is_causal: bool = False, *, workspace=None) -> torch.Tensor:
     """Compact mask_id (None = dense) into a reusable plan held in the returned workspace."""
     B, H, N, d = q.shape
     m = _mask_arg(mask_id, q) if mask_id is not None else None
     ws, wp, wn = _ws(q, workspace)
-    _check(lib().block_sparse_attn_plan(m.data_ptr() if m is not None else None, _shape_of(q), wp, wn,
-                                        _stream(q)))
+    _check(lib().block_sparse_attn_plan(m.data_ptr() if m is not None else None, _shape_of(q),
+                                        int(bool(is_causal)), wp, wn, _stream(q)))
     return ws
 
 
-def block_sparse_attn_apply(q, k, v, workspace, *, out=None):
+def block_sparse_attn_apply(q, k, v, workspace, is_causal: bool = False, *, out=None):
     """Attention over the plan held in `workspace` (from sparse_attn_select,
     sparse_attn_topk or block_sparse_attn_plan on the same shape)."""
     _qkv(q, k, v)
     out = torch.empty_like(q) if out is None else out
     _qkv(q, out)
     _check(lib().block_sparse_attn_apply(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q),
-                                         out.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                         _stream(q)))
+                                         int(bool(is_causal)), out.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel(), _stream(q)))
     return out
 
 

@@ -125,7 +125,7 @@ using namespace bsa;
 
 extern "C" {
 
-int bsa_abi_version(void) { return 1; }
+int bsa_abi_version(void) { return 2; }
 
 const char* bsa_status_string(bsa_status s) {
   switch (s) {
@@ -164,7 +164,7 @@ bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, f
   return BSA_OK;
 }
 
-bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk,
+bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk, int is_causal,
                               uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
   BSA_TRY(check_shape(s));
@@ -178,8 +178,55 @@ bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float t
   const int BH = s.B * s.H;
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
+                         mask_out, w.idx, w.cnt, st),
            "select kernel launch");
+  return BSA_OK;
+}
+
+bsa_status sparse_attn_select_cdf(const void* q, const void* k, bsa_shape s, float threshold,
+                                  uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  if (!(threshold > 0.f) || !(threshold <= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "threshold must lie in (0, 1] (got %g)", static_cast<double>(threshold));
+  if (mask_out == nullptr) return fail(BSA_ERR_INVALID_ARG, "mask_out is NULL");
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+           "cdf select kernel launch");
+  return BSA_OK;
+}
+
+bsa_status sparse_attn_cdf(const void* q, const void* k, const void* v, bsa_shape s, float threshold,
+                           int is_causal, void* out, uint8_t* mask_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  if (is_causal != 0) return fail(BSA_ERR_UNSUPPORTED, "the cdfthreshd mode is non-causal only");
+  BSA_TRY(check_tensor(q, "q"));
+  BSA_TRY(check_tensor(k, "k"));
+  BSA_TRY(check_tensor(v, "v"));
+  BSA_TRY(check_tensor(out, "out"));
+  if (!(threshold > 0.f) || !(threshold <= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "threshold must lie in (0, 1] (got %g)", static_cast<double>(threshold));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+  BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+           "cdf select kernel launch");
+  const char* why = nullptr;
+  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, 0, w.idx, w.cnt, w.status,
+                                   g_timeout_ns.load(), st, &why);
+  if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
   return BSA_OK;
 }
 
@@ -188,7 +235,6 @@ bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bs
                                  size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
   BSA_TRY(check_shape(s));
-  if (is_causal != 0) return fail(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
   BSA_TRY(check_tensor(q, "q"));
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
@@ -198,9 +244,9 @@ bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bs
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
-  BSA_CUDA(launch_compact(mask_id, BH, s.N, w.idx, w.cnt, st), "compaction kernel launch");
+  BSA_CUDA(launch_compact(mask_id, BH, s.N, is_causal != 0, w.idx, w.cnt, st), "compaction kernel launch");
   const char* why = nullptr;
-  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status,
+  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, is_causal != 0, w.idx, w.cnt, w.status,
                                    g_timeout_ns.load(), st, &why);
   if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
   return BSA_OK;
@@ -211,7 +257,6 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
                             void* stream) {
   g_last_error[0] = 0;
   BSA_TRY(check_shape(s));
-  if (is_causal != 0) return fail(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
   BSA_TRY(check_tensor(q, "q"));
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
@@ -224,28 +269,31 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select(w.qbar, w.kbar, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
+                         mask_out, w.idx, w.cnt, st),
            "select kernel launch");
   const char* why = nullptr;
-  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status,
+  cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, is_causal != 0, w.idx, w.cnt, w.status,
                                    g_timeout_ns.load(), st, &why);
   if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
   return BSA_OK;
 }
 
-bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, void* ws, size_t ws_bytes,
-                                  void* stream) {
+bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, int is_causal, void* ws,
+                                  size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
   BSA_TRY(check_shape(s));
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  BSA_CUDA(launch_compact(mask_id, s.B * s.H, s.N, w.idx, w.cnt, st), "compaction kernel launch");
+  BSA_CUDA(launch_compact(mask_id, s.B * s.H, s.N, is_causal != 0, w.idx, w.cnt, st),
+           "compaction kernel launch");
   return BSA_OK;
 }
 
 bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, bsa_shape s,
-                                   void* out, void* ws, size_t ws_bytes, void* stream) {
+                                   int is_causal, void* out, void* ws, size_t ws_bytes,
+                                   void* stream) {
   g_last_error[0] = 0;
   BSA_TRY(check_shape(s));
   BSA_TRY(check_tensor(q, "q"));
@@ -257,8 +305,8 @@ bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   const char* why = nullptr;
-  cudaError_t e = launch_attention(q, k, v, out, s.B * s.H, s.N, s.d, w.idx, w.cnt, w.status,
-                                   g_timeout_ns.load(), st, &why);
+  cudaError_t e = launch_attention(q, k, v, out, s.B * s.H, s.N, s.d, is_causal != 0, w.idx, w.cnt,
+                                   w.status, g_timeout_ns.load(), st, &why);
   if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
   return BSA_OK;
 }

@@ -67,6 +67,7 @@ struct AttnArgs {
   DeviceStatus* status;
   uint64_t timeout_ns;
   int N, Qb, Kb;
+  int causal;        // keys after a row's own position are masked out
   float scale_log2;  // log2(e) / sqrt(d)
 };
 
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(384, 1)
       bar_pfree[2], bar_odone, bar_qkdone;
   __shared__ uint32_t s_tmem;
   __shared__ int s_cnt, s_last, s_fail;
+  __shared__ int s_tail[4];  // the last four kept key blocks (diagonal blocks are among them)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -124,6 +126,8 @@ __global__ void __launch_bounds__(384, 1)
     s_cnt = c;
     s_last = c > 0 ? idx_row[c - 1] : -1;  // the ragged last key block can only be the last kept one
     s_fail = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) s_tail[t] = (c - 4 + t >= 0) ? idx_row[c - 4 + t] : -1;
   }
   __syncthreads();
   const int cnt = s_cnt;
@@ -314,6 +318,24 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < 64; ++c) s[64 + c] = c >= tail ? -INFINITY : s[64 + c];
         }
       }
+      if (a.causal && 2 * j + 1 >= cnt - 4) {
+        // Only the kept blocks 2 qi and 2 qi + 1 straddle the diagonal, and being
+        // the highest kept indices they are among the last four.  Key column c of
+        // block b is visible to row `row` when 64 b + c <= 128 qi + row.
+        const int b0 = s_tail[2 * j - cnt + 4 < 0 ? 0 : 2 * j - cnt + 4];
+        const int b1 = nb == 2 ? s_tail[2 * j + 1 - cnt + 4] : -1;
+        const bool d0 = 2 * j - cnt + 4 >= 0 && b0 >= 2 * qi;
+        const bool d1 = b1 >= 2 * qi;
+        const int lim0 = row - (b0 - 2 * qi) * 64, lim1 = row - (b1 - 2 * qi) * 64;
+        if (d0) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = c > lim0 ? -INFINITY : s[c];
+        }
+        if (d1) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[64 + c] = c > lim1 ? -INFINITY : s[64 + c];
+        }
+      }
       float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
 #pragma unroll
       for (int c = 6; c < 126; c += 4) {
@@ -324,8 +346,12 @@ __global__ void __launch_bounds__(384, 1)
       const float m_new = fmaxf(m_run, rmax * sl2);
       const bool need = m_new > m_run + 8.0f;  // always true for the first pair
       const float m_use = need ? m_new : m_run;
-      const float alpha = ex2_approx(m_run - m_use);  // 0 for the first pair, 1 if no rescale
-      const uint64_t negm = f2_pack(-m_use, -m_use);
+      // A row that has seen no visible key yet (possible only with causal
+      // masking) keeps m = -inf, weight 0 and alpha 1.
+      const bool dead = m_use == -INFINITY;
+      const float alpha = dead ? 1.f : ex2_approx(m_run - m_use);  // 0 for the first pair, 1 if no rescale
+      const float m_ref = dead ? 0.f : m_use;
+      const uint64_t negm = f2_pack(-m_ref, -m_ref);
       // Exponentials of column pairs: x = s * log2(e)/sqrt(d) - m as one f32x2
       // FMA; the pairs selected by C::kPolyPattern on the FMA-pipe polynomial,
       // the rest on MUFU.
@@ -407,9 +433,11 @@ __global__ void __launch_bounds__(384, 1)
       const bool has1 = npairs > 1;  // warpgroup 1 saw at least one pair
       const float m0 = xch[row], m1 = xch[128 + row];
       const float m = has1 ? fmaxf(m0, m1) : m0;
-      const float a0 = ex2_approx(m0 - m);
-      const float a1 = has1 ? ex2_approx(m1 - m) : 0.f;
-      const float inv = 1.f / (xch[256 + row] * a0 + (has1 ? xch[384 + row] * a1 : 0.f));
+      // m = -inf: the row saw no visible key (causal); its output is zero.
+      const float a0 = (m == -INFINITY || m0 == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+      const float a1 = (!has1 || m == -INFINITY || m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+      const float lsum = xch[256 + row] * a0 + (has1 ? xch[384 + row] * a1 : 0.f);
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       const float c0 = a0 * inv, c1 = a1 * inv;
       __nv_bfloat16* orow = out_blk + static_cast<size_t>(row) * D;
 #pragma unroll 1
@@ -540,8 +568,9 @@ cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 }  // namespace
 
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, int BH, int N,
-                             int d, const int16_t* idx, const int32_t* cnt, DeviceStatus* status,
-                             uint64_t timeout_ns, cudaStream_t st, const char** why) {
+                             int d, int causal, const int16_t* idx, const int32_t* cnt,
+                             DeviceStatus* status, uint64_t timeout_ns, cudaStream_t st,
+                             const char** why) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, BH, N, d, kBlockQ) || !make_map(&mk, k, BH, N, d, kBlockK) ||
       !make_map(&mv, v, BH, N, d, kBlockK)) {
@@ -557,6 +586,7 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
   args.N = N;
   args.Qb = (N + kBlockQ - 1) / kBlockQ;
   args.Kb = (N + kBlockK - 1) / kBlockK;
+  args.causal = causal ? 1 : 0;
   args.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
   if (d == 128) return launch_typed<128>(mq, mk, mv, args, BH, st);
   return launch_typed<64>(mq, mk, mv, args, BH, st);

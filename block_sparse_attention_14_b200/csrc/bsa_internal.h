@@ -31,21 +31,32 @@ void set_last_error(const char* msg);
 cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, float* qbar,
                         float* kbar, cudaStream_t st);
 
-// (a3, a4) block scores and top-k; writes mask (optional), idx and cnt.
+// (a3, a4) block scores and top-k; writes mask (optional), idx and cnt.  kkeep is
+// the kept count per row; with causal != 0 each row i instead keeps
+// ceil(topk * E_i) of its E_i = min(2i+2, Kb) eligible blocks.
 cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, int d, int kkeep,
-                          uint8_t* mask_out, int16_t* idx, int32_t* cnt, cudaStream_t st);
+                          float topk, int causal, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
+                          cudaStream_t st);
+
+// cdfthreshd selection: the shortest score-ordered prefix reaching softmax mass
+// `threshold`; writes mask (optional), idx and cnt.
+cudaError_t launch_select_cdf(const float* qbar, const float* kbar, int BH, int N, int d,
+                              float threshold, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
+                              cudaStream_t st);
 
 // (a3) block-score map only: p_out = softmax of the scaled block scores.
 cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, int N, int d,
                                 float* p_out, cudaStream_t st);
 
-// (a4') caller mask (NULL = all ones) -> idx and cnt.
-cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int16_t* idx, int32_t* cnt,
-                           cudaStream_t st);
+// (a4') caller mask (NULL = all ones) -> idx and cnt; causal != 0 drops the
+// blocks past 2i+1 of row i.
+cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int causal, int16_t* idx,
+                           int32_t* cnt, cudaStream_t st);
 
 // (a5, a6) block-sparse attention forward over the idx lists.
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, int BH, int N,
-                             int d, const int16_t* idx, const int32_t* cnt, DeviceStatus* status,
-                             uint64_t timeout_ns, cudaStream_t st, const char** why);
+                             int d, int causal, const int16_t* idx, const int32_t* cnt,
+                             DeviceStatus* status, uint64_t timeout_ns, cudaStream_t st,
+                             const char** why);
 
 }  // namespace bsa

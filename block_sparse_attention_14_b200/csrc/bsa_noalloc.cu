@@ -87,11 +87,12 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
   // The status word must start at zero; everything else is overwritten.
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
       (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
-      (e = launch_select(w.qbar, w.kbar, BH, s.N, s.d, static_cast<int>(kk), mask_out, w.idx, w.cnt,
-                         st)) != cudaSuccess)
+      (e = launch_select(w.qbar, w.kbar, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
+                         w.cnt, st)) != cudaSuccess)
     return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   const char* why = nullptr;
-  e = launch_attention(q, k, v, out, BH, s.N, s.d, w.idx, w.cnt, w.status, wait_timeout_ns(), st, &why);
+  e = launch_attention(q, k, v, out, BH, s.N, s.d, 0, w.idx, w.cnt, w.status, wait_timeout_ns(), st,
+                       &why);
   if (e != cudaSuccess) return reject(BSA_ERR_CUDA, why ? why : cudaGetErrorString(e));
   return BSA_OK;
 }

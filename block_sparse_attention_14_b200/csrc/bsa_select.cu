@@ -219,10 +219,148 @@ __device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, 
   if (lane == 0) *cnt_out = kept;
 }
 
+// cdfthreshd selection of one row by one warp: the shortest prefix, in
+// (score descending, index ascending) order, whose softmax mass reaches tau;
+// at least one block; every block if rounding leaves the total below tau.
+// row[] holds the raw dot products and is overwritten with the probabilities.
+// The largest key T whose mass F(T) = sum of P over keys >= T still reaches
+// tau is found bit by bit (fp32 sums in a fixed lane-then-shuffle order);
+// then every key above T is kept plus the first `need` keys equal to T.
+constexpr int kCdfPer = kMaxKb / 32;
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_fsum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ void warp_cdf_row(float* row, int Kb, float scale, float tau, uint8_t* mask_row,
+                             int16_t* idx_row, int32_t* cnt_out) {
+  const int lane = threadIdx.x & 31;
+  const int nper = (Kb + 31) >> 5;
+  uint32_t key[kCdfPer];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kCdfPer; ++i) {
+    const int j = i * 32 + lane;
+    const bool v = i < nper && j < Kb;
+    key[i] = v ? float_key(row[j]) : 0u;  // 0 is below every real key
+    if (v) mx = fmaxf(mx, row[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float z = 0.f;
+  for (int j = lane; j < Kb; j += 32) {
+    const float e = expf((row[j] - mx) * scale);
+    row[j] = e;
+    z += e;
+  }
+  const float inv = 1.f / warp_fsum(z);
+  for (int j = lane; j < Kb; j += 32) row[j] *= inv;
+  __syncwarp();
+  auto mass_at_or_above = [&](uint32_t cand) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < kCdfPer; ++i)
+      if (i < nper && key[i] >= cand) m += row[i * 32 + lane];
+    return warp_fsum(m);
+  };
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    if (mass_at_or_above(cand) >= tau) T = cand;
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  int kept = 0;
+  if (T == 0) {  // the whole row's mass stays below tau: keep every block
+    for (int j = lane; j < Kb; j += 32) {
+      idx_row[j] = static_cast<int16_t>(j);
+      if (mask_row != nullptr) mask_row[j] = 1;
+    }
+    if (lane == 0) *cnt_out = Kb;
+    return;
+  }
+  float above = 0.f, p_eq = 0.f;
+  int n_eq = 0;
+#pragma unroll
+  for (int i = 0; i < kCdfPer; ++i) {
+    if (i < nper) {
+      if (key[i] > T) above += row[i * 32 + lane];
+      if (key[i] == T) {
+        p_eq = row[i * 32 + lane];
+        ++n_eq;
+      }
+    }
+  }
+  above = warp_fsum(above);
+  p_eq = fmaxf(p_eq, __shfl_xor_sync(0xffffffffu, p_eq, 16));
+  p_eq = fmaxf(p_eq, __shfl_xor_sync(0xffffffffu, p_eq, 8));
+  p_eq = fmaxf(p_eq, __shfl_xor_sync(0xffffffffu, p_eq, 4));
+  p_eq = fmaxf(p_eq, __shfl_xor_sync(0xffffffffu, p_eq, 2));
+  p_eq = fmaxf(p_eq, __shfl_xor_sync(0xffffffffu, p_eq, 1));
+  n_eq = warp_sum(n_eq);
+  int need = p_eq > 0.f ? static_cast<int>(ceilf((tau - above) / p_eq)) : n_eq;
+  need = max(1, min(n_eq, need));
+  int eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < kCdfPer; ++i) {
+    if (i >= nper) break;
+    const int j = i * 32 + lane;
+    const uint32_t u = key[i];
+    const bool valid = j < Kb;
+    const bool eq = valid && u == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool keep = valid && (u > T || (eq && eq_seen + __popc(eqb & lt) < need));
+    eq_seen += __popc(eqb);
+    const unsigned kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) idx_row[kept + __popc(kb & lt)] = static_cast<int16_t>(j);
+    if (mask_row != nullptr && valid) mask_row[j] = keep ? 1 : 0;
+    kept += __popc(kb);
+  }
+  if (lane == 0) *cnt_out = kept;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_cdf_kernel(const float* __restrict__ qbar,
+                                                                 const float* __restrict__ kbar,
+                                                                 int Qb, int Kb, float scale,
+                                                                 float tau,
+                                                                 uint8_t* __restrict__ mask_out,
+                                                                 int16_t* __restrict__ idx,
+                                                                 int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(16) float smem[];
+  float* sq = smem;
+  float* sc = sq + kSelG * D;
+  const int bh = blockIdx.y;
+  const int i0 = blockIdx.x * kSelG;
+  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
+  const int w = threadIdx.x >> 5;
+  const int i = i0 + w;
+  if (i >= Qb) return;
+  const size_t row = static_cast<size_t>(bh) * Qb + i;
+  warp_cdf_row(sc + w * Kb, Kb, scale, tau, mask_out ? mask_out + row * Kb : nullptr,
+               idx + row * Kb, cnt + row);
+}
+
+// Kept count for a fraction of E blocks: clamp(ceil(topk * E), 1, E) in double
+// precision on the float value of topk (the host computes the same for the
+// non-causal case).
+__device__ __forceinline__ int keep_count_dev(float topk, int E) {
+  int k = static_cast<int>(ceil(static_cast<double>(topk) * static_cast<double>(E)));
+  return max(1, min(E, k));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ qbar,
                                                              const float* __restrict__ kbar,
-                                                             int Qb, int Kb, int kk,
+                                                             int Qb, int Kb, int kk, float topk,
+                                                             int causal,
                                                              uint8_t* __restrict__ mask_out,
                                                              int16_t* __restrict__ idx,
                                                              int32_t* __restrict__ cnt) {
@@ -237,8 +375,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   const int i = i0 + w;
   if (i >= Qb) return;
   const size_t row = static_cast<size_t>(bh) * Qb + i;
-  warp_topk_row(sc + w * Kb, Kb, kk, hist + w * 256,
-                mask_out ? mask_out + row * Kb : nullptr, idx + row * Kb, cnt + row);
+  // Causal: query block i may use key blocks 0 .. 2i+1 only; top-k runs over those.
+  const int Ke = causal ? min(2 * i + 2, Kb) : Kb;
+  const int k_row = causal ? keep_count_dev(topk, Ke) : kk;
+  uint8_t* mrow = mask_out ? mask_out + row * Kb : nullptr;
+  warp_topk_row(sc + w * Kb, Ke, k_row, hist + w * 256, mrow, idx + row * Kb, cnt + row);
+  if (mrow != nullptr)
+    for (int j = Ke + (threadIdx.x & 31); j < Kb; j += 32) mrow[j] = 0;
 }
 
 template <int D>
@@ -273,18 +416,21 @@ __global__ void __launch_bounds__(kSelThreads) block_scores_kernel(const float* 
 // ----------------------------------------------------------------- compaction
 // One warp per (b, h, i) row: kept block indices in ascending order.
 __global__ void __launch_bounds__(256) compact_kernel(const uint8_t* __restrict__ mask, int rows,
-                                                      int Kb, int16_t* __restrict__ idx,
+                                                      int Qb, int Kb, int causal,
+                                                      int16_t* __restrict__ idx,
                                                       int32_t* __restrict__ cnt) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+  // Causal: blocks past 2i+1 hold only later keys and are dropped.
+  const int limit = causal ? min(2 * (row % Qb) + 2, Kb) : Kb;
   const uint8_t* m = mask ? mask + static_cast<size_t>(row) * Kb : nullptr;
   int16_t* out = idx + static_cast<size_t>(row) * Kb;
   const unsigned lt = (1u << lane) - 1u;
   int kept = 0;
   for (int base = 0; base < Kb; base += 32) {
     const int j = base + lane;
-    const bool keep = (j < Kb) && (m == nullptr || m[j] != 0);
+    const bool keep = (j < limit) && (m == nullptr || m[j] != 0);
     const unsigned b = __ballot_sync(0xffffffffu, keep);
     if (keep) out[kept + __popc(b & lt)] = static_cast<int16_t>(j);
     kept += __popc(b);
@@ -316,7 +462,8 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
 }
 
 cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, int d, int kk,
-                          uint8_t* mask_out, int16_t* idx, int32_t* cnt, cudaStream_t st) {
+                          float topk, int causal, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
+                          cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   dim3 grid((Qb + kSelG - 1) / kSelG, BH);
@@ -326,12 +473,39 @@ cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, i
     e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    select_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, mask_out, idx, cnt);
+    select_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, topk, causal, mask_out,
+                                                        idx, cnt);
   } else {
     e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    select_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, mask_out, idx, cnt);
+    select_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, topk, causal, mask_out,
+                                                       idx, cnt);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_cdf(const float* qbar, const float* kbar, int BH, int N, int d,
+                              float threshold, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
+                              cudaStream_t st) {
+  const int Qb = (N + kBlockQ - 1) / kBlockQ;
+  const int Kb = (N + kBlockK - 1) / kBlockK;
+  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
+  const size_t smem = select_smem(d, Kb, false);
+  const float scale = 1.0f / sqrtf(static_cast<float>(d));
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(select_cdf_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    select_cdf_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, threshold,
+                                                            mask_out, idx, cnt);
+  } else {
+    e = cudaFuncSetAttribute(select_cdf_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    select_cdf_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, threshold,
+                                                           mask_out, idx, cnt);
   }
   return cudaGetLastError();
 }
@@ -358,12 +532,12 @@ cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int16_t* idx, int32_t* cnt,
-                           cudaStream_t st) {
+cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int causal, int16_t* idx,
+                           int32_t* cnt, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int rows = BH * Qb;
-  compact_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mask, rows, Kb, idx, cnt);
+  compact_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mask, rows, Qb, Kb, causal, idx, cnt);
   return cudaGetLastError();
 }
 

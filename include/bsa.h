@@ -49,7 +49,8 @@ extern "C" {
 typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment, topk or workspace size */
-  BSA_ERR_UNSUPPORTED = 2, /* is_causal != 0 */
+  BSA_ERR_UNSUPPORTED = 2, /* an unsupported mode combination (is_causal with cdfthreshd or the
+                              no-allocation call) */
   BSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   BSA_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out */
 } bsa_status;
@@ -62,7 +63,7 @@ typedef struct {
 } bsa_shape;
 
 /* Version of this ABI (incremented on incompatible changes). */
-int bsa_abi_version(void);
+int bsa_abi_version(void);  /* 2: is_causal added to select / plan / apply */
 
 /* Human-readable name of a status code (static string). */
 const char* bsa_status_string(bsa_status s);
@@ -88,23 +89,47 @@ bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, f
  * kk = clamp(ceil(topk * Kb), 1, Kb) ones per (b, h, i) row: the kk key blocks
  * with the largest block score, equal scores going to the lower block index.
  * kk is evaluated in double precision on the float value of topk.
- * topk must lie in (0, 1]. */
-bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk,
+ * topk must lie in (0, 1].  With is_causal != 0, row i chooses only among its
+ * E_i = min(2 i + 2, Kb) causally eligible key blocks (blocks that hold a key
+ * at or before some row of query block i) and keeps clamp(ceil(topk * E_i), 1,
+ * E_i) of them; the other entries of the row are 0. */
+bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float topk, int is_causal,
                               uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream);
+
+/* cdfthreshd selection (the "--mode cdfthreshd" option next to "topk" on
+ * "SpargeAttention Documentation"; the pages print no formula, so this is a
+ * reading): per (b, h, i) row, order the key blocks by block score descending
+ * (equal scores: lower index first) and keep the shortest prefix whose
+ * softmax mass reaches `threshold` (its float value, in (0, 1]); at least one
+ * block; every block if rounding leaves the row's total mass below threshold.
+ * Writes mask_out (device, uint8 [B, H, Qb, Kb]) and the plan in ws. */
+bsa_status sparse_attn_select_cdf(const void* q, const void* k, bsa_shape s, float threshold,
+                                  uint8_t* mask_out, void* ws, size_t ws_bytes, void* stream);
+
+/* cdfthreshd selection followed by attention (the fused counterpart of
+ * sparse_attn_topk for the cdfthreshd mode).  mask_out is optional.  This mode
+ * is non-causal only: is_causal != 0 returns BSA_ERR_UNSUPPORTED. */
+bsa_status sparse_attn_cdf(const void* q, const void* k, const void* v, bsa_shape s, float threshold,
+                           int is_causal, void* out, uint8_t* mask_out, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /* Attention over caller-chosen tiles.  mask_id (device, uint8 [B, H, Qb, Kb];
  * NULL means all ones, i.e. dense attention) selects the kept 128 x 64 tiles.
  * For every query row r of block i: out[r] = sum over kept tiles j and key rows
  * c < N of block j of softmax_c(q_r . k_c / sqrt(d)) v_c, the softmax taken
  * over the union of the kept keys.  A query block that keeps no key block gets
- * an all-zero output.  Rows >= N are never written.  is_causal must be 0. */
+ * an all-zero output.  Rows >= N are never written.  With is_causal != 0 only
+ * keys c <= r take part (mask entries past block 2 i + 1 are ignored and the
+ * two diagonal blocks are masked element by element); a row left without any
+ * key gets a zero output. */
 bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bsa_shape s,
                                  const uint8_t* mask_id, int is_causal, void* out,
                                  void* ws, size_t ws_bytes, void* stream);
 
 /* Selection followed by attention in one call (three kernels on one stream,
  * no host synchronisation).  mask_out is optional (NULL: not written); when
- * given it receives the selection mask of sparse_attn_select. */
+ * given it receives the selection mask of sparse_attn_select.  is_causal has
+ * the meaning of sparse_attn_select and block_sparse_attn_fwd. */
 bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_shape s, float topk,
                             int is_causal, void* out, uint8_t* mask_out, void* ws,
                             size_t ws_bytes, void* stream);
@@ -114,14 +139,16 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
  * sparse_attn_select, sparse_attn_topk or block_sparse_attn_plan leave in ws
  * form a reusable plan.  block_sparse_attn_plan compacts a caller mask
  * (NULL = all ones) into ws without running attention. */
-bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, void* ws, size_t ws_bytes,
-                                  void* stream);
+bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, int is_causal, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Attention over the plan currently held in ws (see block_sparse_attn_plan);
  * same output contract as block_sparse_attn_fwd.  The plan must have been
- * made for the same shape; ws is not modified apart from its status word. */
+ * made for the same shape and the same is_causal; ws is not modified apart
+ * from its status word. */
 bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, bsa_shape s,
-                                   void* out, void* ws, size_t ws_bytes, void* stream);
+                                   int is_causal, void* out, void* ws, size_t ws_bytes,
+                                   void* stream);
 
 /* No-allocation variant of sparse_attn_topk (same arguments minus the
  * workspace; same kernels, same results).  The pages have no counterpart: this

@@ -67,3 +67,15 @@ def oracle_rows(q, k, v, mask_np: np.ndarray, b: int, h: int, blocks, cache=None
 def gpu_rows(out: torch.Tensor, b: int, h: int, blocks, N: int):
     o = out[b, h].float().cpu().numpy()
     return [o[i * 128:min(N, (i + 1) * 128)] for i in blocks]
+
+
+def compare_cdf_masks(mask_gpu: torch.Tensor, mask_ref: np.ndarray, P_ref: np.ndarray, tau: float):
+    """cdfthreshd masks: rows may differ only where the decision is not determined
+    at the inputs' precision (O.cdf_exempt_rows).  Every GPU row keeps at least one
+    block.  Returns (non-exempt mismatching rows, exempt rows)."""
+    mg = mask_gpu.cpu().numpy().astype(np.uint8)
+    assert mg.shape == mask_ref.shape
+    assert np.all(mg.sum(-1) >= 1)
+    diff = np.any(mg != mask_ref, axis=-1)
+    ex = O.cdf_exempt_rows(P_ref, tau)
+    return int((diff & ~ex).sum()), int(ex.sum())

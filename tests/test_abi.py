@@ -24,7 +24,7 @@ def test_library_exports_every_declared_function():
     L = bsa.lib()
     for n in names:
         assert hasattr(L, n), n
-    assert L.bsa_abi_version() == 1
+    assert L.bsa_abi_version() == 2
 
 
 def test_status_strings():
@@ -60,7 +60,6 @@ def _call_topk(shape, topk=0.5, is_causal=0, q=256, k=256, v=256, out=256, ws=51
     (dict(shape=(1, 1, 128, 64), topk=0.0), 1),
     (dict(shape=(1, 1, 128, 64), topk=1.5), 1),
     (dict(shape=(1, 1, 128, 64), topk=float("nan")), 1),
-    (dict(shape=(1, 1, 128, 64), is_causal=1), 2),
     (dict(shape=(1, 1, 128, 64), q=None), 1),
     (dict(shape=(1, 1, 128, 64), v=264), 1),        # unaligned pointer
     (dict(shape=(1, 1, 128, 64), ws=None), 1),
@@ -76,10 +75,15 @@ def test_other_calls_reject_bad_arguments():
     L = bsa.lib()
     s = bsa.Shape(1, 2, 300, 64)
     n = L.bsa_workspace_bytes(s)
-    assert L.block_sparse_attn_fwd(256, 256, 256, s, None, 1, 256, 512, n, None) == 2
     assert L.block_sparse_attn_fwd(256, 256, 256, s, None, 0, None, 512, n, None) == 1
-    assert L.sparse_attn_select(256, 256, s, 0.5, None, 512, n, None) == 1
-    assert L.sparse_attn_select(256, 256, s, -1.0, 1024, 512, n, None) == 1
+    assert L.sparse_attn_select(256, 256, s, 0.5, 0, None, 512, n, None) == 1
+    assert L.sparse_attn_select(256, 256, s, -1.0, 1, 1024, 512, n, None) == 1
+    assert L.block_sparse_attn_plan(None, bsa.Shape(1, 1, 64, 96), 0, 512, n, None) == 1
+    assert L.block_sparse_attn_apply(256, 256, 256, s, 0, None, 512, n, None) == 1
+    na = L.sparse_attn_topk_noalloc
+    na.restype = ctypes.c_int
+    na.argtypes = [ctypes.c_void_p] * 3 + [bsa.Shape, ctypes.c_float, ctypes.c_int] + [ctypes.c_void_p] * 3
+    assert na(256, 256, 256, s, 0.5, 1, 256, None, None) == 2  # the no-allocation call is non-causal
     assert L.sparse_attn_block_scores(256, 256, s, None, 512, n, None) == 1
     assert L.sparse_attn_block_scores(256, 256, bsa.Shape(1, 2, 300, 32), 1024, 512, n, None) == 1
     assert L.bsa_last_device_status(None, None) == 1
@@ -99,3 +103,14 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         bsa.sparse_attn_topk(q, q, q, 0.5)
+
+
+def test_cdf_calls_reject_bad_thresholds():
+    L = bsa.lib()
+    s = bsa.Shape(1, 2, 300, 64)
+    n = L.bsa_workspace_bytes(s)
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        assert L.sparse_attn_select_cdf(256, 256, s, bad, 1024, 512, n, None) == 1
+        assert L.sparse_attn_cdf(256, 256, 256, s, bad, 0, 256, None, 512, n, None) == 1
+    assert L.sparse_attn_cdf(256, 256, 256, s, 0.9, 1, 256, None, 512, n, None) == 2
+    assert L.sparse_attn_select_cdf(256, 256, s, 0.9, None, 512, n, None) == 1

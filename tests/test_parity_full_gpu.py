@@ -104,3 +104,17 @@ def test_wan14b_caller_mask(density):
 
 def test_hunyuan13b_fused_topk01():
     _fused_case("hunyuan13b", 0.1, heads=[0, 5, 11, 17, 23], n_random=6)
+
+
+def test_wan13b_fused_cdf09():
+    from tests.parity import compare_cdf_masks
+
+    wl, qkv_cpu, (q, k, v) = _inputs("wan13b")
+    ws = bsa.make_workspace(wl.B, wl.H, wl.N, wl.d)
+    out, mask = bsa.sparse_attn_cdf(q, k, v, 0.9, return_mask=True, workspace=ws)
+    bsa.last_device_status(ws)
+    mref, P = O.cdf_mask(_oracle_select("wan13b", 1.0)[1], 0.9), _oracle_select("wan13b", 1.0)[1]
+    bad, _ = compare_cdf_masks(mask, mref, P, 0.9)
+    assert bad == 0
+    agree = np.all(mask.cpu().numpy() == mref, axis=-1)
+    _check_rows(out, wl, qkv_cpu, mref, agree, range(wl.H), 3, seed=90)

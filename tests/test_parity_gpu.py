@@ -155,11 +155,88 @@ def test_no_writes_outside_output_and_deterministic(cuda_device):
     assert torch.equal(first, out)
 
 
-def test_causal_rejected_and_status_ok(cuda_device):
+def test_status_ok_after_a_normal_call(cuda_device):
     q, k, v = _cuda(*_qkv(1, 1, 256, 64, seed=1))
-    with pytest.raises(bsa.BsaError) as e:
-        bsa.sparse_attn_topk(q, k, v, 0.5, is_causal=True)
-    assert e.value.status == 2
     ws = bsa.make_workspace(1, 1, 256, 64)
     bsa.sparse_attn_topk(q, k, v, 0.5, workspace=ws)
     bsa.last_device_status(ws)  # raises on a recorded timeout
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.sparse_attn_cdf(q, k, v, 0.9, is_causal=True)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 1024, 64), (1, 2, 300, 128), (2, 2, 4113, 128), (1, 1, 65, 64)])
+def test_causal_dense_matches_oracle(B, H, N, d, cuda_device):
+    q, k, v = _qkv(B, H, N, d, seed=N + 3 * d, scale=1.5)
+    out = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), None, is_causal=True)
+    torch.cuda.synchronize()
+    Qb, Kb = O.block_counts(N)
+    ref = O.block_sparse_attention(q, k, v, np.ones((B, H, Qb, Kb), np.uint8), causal=True)
+    assert_close(out.float().cpu().numpy(), ref, f"causal dense {B,H,N,d}")
+
+
+@pytest.mark.parametrize("N,d,density", [(2000, 128, 0.5), (1537, 64, 0.3)])
+def test_causal_caller_mask_matches_oracle(N, d, density, cuda_device):
+    B, H = 1, 3
+    q, k, v = _qkv(B, H, N, d, seed=11 * N + d, scale=2.0)
+    Qb, Kb = O.block_counts(N)
+    g = torch.Generator().manual_seed(N + 5)
+    mask = (torch.rand(B, H, Qb, Kb, generator=g) < density).to(torch.uint8)
+    mask[0, 0, 2] = 0
+    mask[0, 0, 2, 5] = 1          # only the second diagonal block: rows 256..319 see nothing
+    mask[0, 1, 3] = 0
+    mask[0, 1, 3, 7] = 1
+    mask[0, 1, 3, 9] = 1          # an ineligible block, ignored under causal attention
+    out = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), mask.cuda(), is_causal=True)
+    torch.cuda.synchronize()
+    ref = O.block_sparse_attention(q, k, v, mask.numpy(), causal=True)
+    got = out.float().cpu().numpy()
+    assert np.all(got[0, 0, 256:320] == 0)
+    assert_close(got, ref, f"causal mask {N,d,density}")
+
+
+@pytest.mark.parametrize("N,d,topk", [(3000, 128, 0.5), (2500, 64, 0.3), (777, 128, 0.2)])
+def test_causal_fused_topk_matches_oracle(N, d, topk, cuda_device):
+    wl = W.custom("ct", B=1, H=3, d=d, N=N, seed=N + 7)
+    q, k, v = W.make_qkv(wl)
+    qc, kc, vc = _cuda(q, k, v)
+    out, mask = bsa.sparse_attn_topk(qc, kc, vc, topk, is_causal=True, return_mask=True)
+    m2 = bsa.sparse_attn_select(qc, kc, topk, is_causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, m2)
+    mref, P = O.select(q, k, topk, causal=True)
+    mg = mask.cpu().numpy()
+    Qb, Kb = wl.Qb, wl.Kb
+    for i in range(Qb):  # per-row k and eligibility; rows may differ only within the tie band
+        E = O.causal_block_limit(i, Kb)
+        kk = O.keep_count(topk, E)
+        assert np.all(mg[:, :, i, E:] == 0)
+        assert np.all(mg[:, :, i].sum(-1) == kk)
+        diff = np.any(mg[:, :, i] != mref[:, :, i], axis=-1)
+        ex = O.tie_exempt_rows(P[:, :, i:i + 1, :E], kk)[:, :, 0]
+        assert not np.any(diff & ~ex)
+    ref = O.block_sparse_attention(q, k, v, mref, causal=True)
+    same = np.all(mg == mref, axis=-1)
+    rows = np.repeat(same, 128, axis=2)[:, :, :N]
+    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"causal topk {N,d,topk}")
+
+
+@pytest.mark.parametrize("N,d,tau", [(3000, 128, 0.5), (3000, 128, 0.9), (2500, 64, 0.95), (777, 128, 0.3),
+                                     (4096, 64, 1.0)])
+def test_cdf_selection_and_attention_match_oracle(N, d, tau, cuda_device):
+    from tests.parity import compare_cdf_masks
+
+    wl = W.custom("cdf", B=1, H=3, d=d, N=N, seed=N + 1)
+    q, k, v = W.make_qkv(wl)
+    qc, kc, vc = _cuda(q, k, v)
+    m1 = bsa.sparse_attn_select_cdf(qc, kc, tau)
+    out, m2 = bsa.sparse_attn_cdf(qc, kc, vc, tau, return_mask=True)
+    torch.cuda.synchronize()
+    assert torch.equal(m1, m2)
+    mref, P = O.select_cdf(q, k, tau)
+    bad, _ = compare_cdf_masks(m1, mref, P, tau)
+    assert bad == 0
+    ref = O.block_sparse_attention(q, k, v, mref)
+    same = np.all(m1.cpu().numpy() == mref, axis=-1)
+    rows = np.repeat(same, 128, axis=2)[:, :, :N]
+    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"cdf {N,d,tau}")
