@@ -31,7 +31,7 @@ import torch
 __all__ = [
     "BsaError", "sparse_attn_topk", "block_sparse_attn_fwd", "sparse_attn_select",
     "sparse_attn_block_scores", "sparse_attn_select_cdf", "sparse_attn_cdf", "workspace_bytes", "make_workspace", "last_device_status",
-    "set_wait_timeout_ns", "block_sparse_attn_plan", "block_sparse_attn_apply", "block_counts", "keep_count", "library_path", "lib",
+    "set_wait_timeout_ns", "token_permutation", "permute_tokens", "block_sparse_attn_plan", "block_sparse_attn_apply", "block_counts", "keep_count", "library_path", "lib",
 ]
 
 BLOCK_Q = 128
@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.block_sparse_attn_plan.argtypes = [vp, Shape, i32, vp, sz, vp]
         L.block_sparse_attn_apply.restype = i32
         L.block_sparse_attn_apply.argtypes = [vp, vp, vp, Shape, i32, vp, vp, sz, vp]
+        L.bsa_token_permutation.restype = i32
+        L.bsa_token_permutation.argtypes = [i32, i32, i32, i32, i32, vp]
+        L.bsa_permute_tokens.restype = i32
+        L.bsa_permute_tokens.argtypes = [vp, vp, Shape, vp, i32, vp]
         L.bsa_last_device_status.restype = i32
         L.bsa_last_device_status.argtypes = [vp, vp]
         L.bsa_set_wait_timeout_ns.restype = None
@@ -283,6 +287,30 @@ def block_sparse_attn_apply(q, k, v, workspace, is_causal: bool = False, *, out=
     _check(lib().block_sparse_attn_apply(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q),
                                          int(bool(is_causal)), out.data_ptr(), workspace.data_ptr(),
                                          workspace.numel(), _stream(q)))
+    return out
+
+
+REORDER_MODES = {"raster": 0, "cube": 1, "morton": 2}
+
+
+def token_permutation(T: int, Hg: int, Wg: int, text: int = 0, mode: str = "cube") -> torch.Tensor:
+    """perm[new] = old for a [text | T x Hg x Wg video] sequence (host int32 tensor)."""
+    perm = torch.empty(text + T * Hg * Wg, dtype=torch.int32)
+    _check(lib().bsa_token_permutation(T, Hg, Wg, text, REORDER_MODES[mode], perm.data_ptr()))
+    return perm
+
+
+def permute_tokens(x: torch.Tensor, perm: torch.Tensor, inverse: bool = False, *, out=None) -> torch.Tensor:
+    """Reorder the token axis of a contiguous CUDA bf16 [B, H, N, d] tensor by perm
+    (a CUDA int32 permutation of 0..N-1): out[:, :, n] = x[:, :, perm[n]], or the
+    inverse with inverse=True."""
+    _qkv(x)
+    if not (perm.is_cuda and perm.dtype == torch.int32 and perm.numel() == x.shape[2] and perm.is_contiguous()):
+        raise ValueError("perm must be a contiguous CUDA int32 tensor of N entries")
+    out = torch.empty_like(x) if out is None else out
+    _qkv(x, out)
+    _check(lib().bsa_permute_tokens(x.data_ptr(), out.data_ptr(), _shape_of(x), perm.data_ptr(),
+                                    int(bool(inverse)), _stream(x)))
     return out
 
 

@@ -170,6 +170,25 @@ bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
                                     float topk, int is_causal, void* out, uint8_t* mask_out,
                                     void* stream);
 
+/* Token reordering (after the AB-Attention README's "Optional cube layout" and
+ * the Morton3D ordering of the LightX2V page "Sol-Attn on Wan2.1"): writes
+ * perm_out (host int32, text + T*Hg*Wg entries), perm[new] = old, for a
+ * sequence of `text` tokens followed by a T x Hg x Wg video grid in raster
+ * order.  Text tokens stay first and in place.  mode 0: raster (identity);
+ * mode 1: 4 x 4 x 4 cubes, ordered by (t/4, h/4, w/4, t%4, h%4, w%4), cubes
+ * clipped at the edges; mode 2: Morton3D, the key interleaving the bits of
+ * (t, h, w).  Host only; no device memory is touched. */
+bsa_status bsa_token_permutation(int T, int Hg, int Wg, int text, int mode, int32_t* perm_out);
+
+/* Applies a token permutation to a contiguous [B, H, N, d] bf16 tensor:
+ * dst[b, h, n] = src[b, h, perm[n]] (inverse = 0), or dst[b, h, perm[n]] =
+ * src[b, h, n] (inverse != 0, undoing the first).  perm is a device int32
+ * array of N entries that must be a permutation of 0..N-1 (not checked); src
+ * and dst are distinct 16-byte aligned device buffers; d is a multiple of 8.
+ * Asynchronous on `stream`. */
+bsa_status bsa_permute_tokens(const void* src, void* dst, bsa_shape s, const int32_t* perm, int inverse,
+                              void* stream);
+
 /* Synchronises `stream`, then reports what the kernels of the last call that
  * used `ws` recorded: BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out), or
  * BSA_ERR_CUDA if the stream holds an error. */

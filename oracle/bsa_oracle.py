@@ -285,3 +285,49 @@ def tie_exempt_rows(P: np.ndarray, k: int, rel: float = 1e-6) -> np.ndarray:
     s = -np.sort(-P, axis=-1)
     pk, pk1 = s[..., k - 1], s[..., k]
     return (pk - pk1) < rel * pk
+
+
+# ------------------------------------------------------------ token reordering
+def token_permutation(T: int, Hg: int, Wg: int, text: int, mode: str) -> np.ndarray:
+    """perm[new_position] = old_position for a [text | T x Hg x Wg video] sequence.
+
+    The AB-Attention README ("Optional cube layout") groups video tokens into
+    4 x 4 x 4 spatiotemporal cubes; the LightX2V page ("Sol-Attn on Wan2.1")
+    applies a Morton3D ordering.  Readings: text tokens stay first and in place;
+    "cube" orders video tokens by (t//4, h//4, w//4, t%4, h%4, w%4), cubes
+    clipped at the grid edges; "morton" orders them by the Z-order key that
+    interleaves the bits of (t, h, w) (t highest in each bit triple), ties
+    impossible; "raster" is the identity.
+    """
+    nv = T * Hg * Wg
+    m = np.arange(nv)
+    t, h, w = m // (Hg * Wg), (m // Wg) % Hg, m % Wg
+    if mode == "raster":
+        order = m
+    elif mode == "cube":
+        order = np.lexsort((w % 4, h % 4, t % 4, w // 4, h // 4, t // 4))
+    elif mode == "morton":
+        key = np.zeros(nv, dtype=np.int64)
+        for b in range(21):
+            key |= ((t >> b) & 1) << (3 * b + 2)
+            key |= ((h >> b) & 1) << (3 * b + 1)
+            key |= ((w >> b) & 1) << (3 * b)
+        order = np.argsort(key, kind="stable")
+    else:
+        raise ValueError(mode)
+    return np.concatenate([np.arange(text), text + order]).astype(np.int64)
+
+
+def kept_mass(q, k, mask, b: int, h: int, blocks) -> np.ndarray:
+    """Share of each sampled row's dense softmax mass that falls in its kept key
+    blocks (1.0 = the selection loses nothing), for the listed query blocks."""
+    qh, kh = to_f64(q[b, h]), to_f64(k[b, h])
+    N, d = qh.shape
+    out = []
+    for i in blocks:
+        lo, hi = i * BLOCK_Q, min((i + 1) * BLOCK_Q, N)
+        S = qh[lo:hi] @ kh.T / math.sqrt(d)
+        E = np.exp(S - S.max(axis=1, keepdims=True))
+        cols = kept_key_columns(mask[b, h, i], N)
+        out.append(E[:, cols].sum(axis=1) / E.sum(axis=1))
+    return np.concatenate(out)

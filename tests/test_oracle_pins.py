@@ -453,3 +453,44 @@ def test_causal_topk_matches_brute_force_over_eligible_blocks():
             kk = O.keep_count(topk, E)
             assert m[0, 0, i, E:].sum() == 0
             assert tuple(np.flatnonzero(m[0, 0, i])) == _brute_topk(list(P[0, 0, i, :E]), kk)
+
+
+# --------------------------------------------------------- token reordering
+def test_token_permutations_hand_worked():
+    # 1 x 2 x 8 grid, no text: cubes of 4 x 4 x 4 clip to 1 x 2 x 4, so the cube
+    # order takes columns 0-3 of both rows, then columns 4-7 of both rows.
+    p = O.token_permutation(1, 2, 8, 0, "cube")
+    assert list(p) == [0, 1, 2, 3, 8, 9, 10, 11, 4, 5, 6, 7, 12, 13, 14, 15]
+    # Morton on a 1 x 2 x 4 grid: key interleaves (h, w) bits -> (0,0)(0,1)(1,0)(1,1)(0,2)(0,3)(1,2)(1,3)
+    p = O.token_permutation(1, 2, 4, 0, "morton")
+    assert list(p) == [0, 1, 4, 5, 2, 3, 6, 7]
+    p = O.token_permutation(2, 3, 5, 4, "raster")
+    assert list(p) == list(range(34))
+
+
+@pytest.mark.parametrize("mode", ["cube", "morton"])
+def test_token_permutation_is_a_bijection_keeping_text_first(mode):
+    for T, Hg, Wg, text in [(21, 45, 80, 0), (13, 30, 45, 226), (1, 1, 7, 3), (5, 9, 6, 0)]:
+        p = O.token_permutation(T, Hg, Wg, text, mode)
+        assert sorted(p.tolist()) == list(range(text + T * Hg * Wg))
+        assert list(p[:text]) == list(range(text))
+
+
+def test_cube_blocks_are_spatially_compact():
+    # every aligned run of 64 tokens inside full cubes spans a 4 x 4 x 4 box
+    T, Hg, Wg = 8, 8, 8
+    p = O.token_permutation(T, Hg, Wg, 0, "cube")
+    for s0 in range(0, T * Hg * Wg, 64):
+        m = p[s0:s0 + 64]
+        t, h, w = m // 64, (m // 8) % 8, m % 8
+        assert np.ptp(t) == 3 and np.ptp(h) == 3 and np.ptp(w) == 3
+
+
+def test_kept_mass_is_one_for_dense_and_below_one_for_sparse():
+    rng = _rng(41)
+    q, k = rng.normal(size=(1, 1, 300, 16)) * 2, rng.normal(size=(1, 1, 300, 16)) * 2
+    ones = np.ones((1, 1, 3, 5), np.uint8)
+    np.testing.assert_allclose(O.kept_mass(q, k, ones, 0, 0, [0, 2]), 1.0, atol=1e-12)
+    half = ones.copy(); half[..., 1::2] = 0
+    km = O.kept_mass(q, k, half, 0, 0, [0, 1, 2])
+    assert np.all(km < 1) and np.all(km > 0)
