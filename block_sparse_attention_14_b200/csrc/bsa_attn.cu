@@ -18,8 +18,9 @@
 // block) in the S buffer of warpgroup w = j % 2.  The warpgroup copies S into
 // registers and releases the buffer at once, so the tensor core computes
 // S_{j+2} while the exponentials of pair j run.  P (bf16) goes to a per-
-// warpgroup shared-memory tile in the K-major 128-byte-swizzled layout, and
-// O_w += P V accumulates in TMEM.  Each warpgroup keeps its own running max,
+// warpgroup tile -- in TMEM for d = 64, where P.V then reads its A operand
+// from TMEM; in shared memory (K-major, 128-byte swizzle) for d = 128, whose
+// O accumulators leave no TMEM room -- and O_w += P V accumulates in TMEM.  Each warpgroup keeps its own running max,
 // row sum and O accumulator; the two are merged in the epilogue.
 // The online softmax works in the exp2 domain and only rescales O when the row
 // maximum grows by more than 2^8, which keeps every exponent <= 2^8 and is
@@ -38,13 +39,14 @@ namespace bsa {
 namespace {
 
 // Column pairs c with bit (c % 8) set use the FMA-pipe exp2 polynomial; the
-// others use MUFU ex2.  One pair in four (0x88) balanced MUFU throughput
-// against issue slots best on B200 (measured against 0, 1/8, 3/8 and 1/2).
+// others use MUFU ex2.  Measured on B200 against 0, 1/8, 1/4, 3/8 and 1/2:
+// d = 128 is fastest with one pair in four (0x88), d = 64 with three in
+// eight (0xA8).
 #ifndef BSA_POLY_PATTERN
 #define BSA_POLY_PATTERN 0x88
 #endif
 #ifndef BSA_POLY_PATTERN_D64
-#define BSA_POLY_PATTERN_D64 0x88
+#define BSA_POLY_PATTERN_D64 0xA8
 #endif
 
 enum WaitSite : uint32_t {
@@ -78,16 +80,21 @@ struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;   // a pair of 64-row key blocks
-  static constexpr int kKSt = (D == 128) ? 2 : 3;
-  static constexpr int kVSt = (D == 128) ? 2 : 3;
-  static constexpr int kPBytes = 128 * 128 * 2;  // one warpgroup's P tile
+  // With d = 64 the P tiles fit in TMEM next to S and O, and P.V reads its A
+  // operand from there; with d = 128 TMEM is full and P goes through shared
+  // memory.
+  static constexpr bool kPTmem = D == 64;
+  static constexpr int kKSt = (D == 128) ? 2 : 4;
+  static constexpr int kVSt = (D == 128) ? 2 : 4;
+  static constexpr int kPBytes = 128 * 128 * 2;  // one warpgroup's P tile (shared memory)
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + kKSt * kKVBytes;
-  static constexpr int kOffP = kOffV + kVSt * kKVBytes;
-  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;  // + alignment slack
-  // TMEM columns: S buffer w at 128 w, O_w at 256 + D w.
+  static constexpr int kOffP = kOffV + kVSt * kKVBytes;  // P tiles, or the epilogue exchange
+  static constexpr int kSmem = kOffP + (kPTmem ? 2048 : 2 * kPBytes) + 1024;  // + alignment slack
+  // TMEM columns: S buffer w at 128 w, O_w at 256 + D w, P_w at 384 + 64 w.
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
+  static constexpr uint32_t kColP = 384;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr unsigned kPolyPattern = (D == 64) ? BSA_POLY_PATTERN_D64 : BSA_POLY_PATTERN;
   static constexpr uint32_t kRegCtl = 56;   // registers per thread, control warpgroup
@@ -262,14 +269,23 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         const int nb = min(2, cnt - 2 * j);
         const uint64_t vd = sw128_desc(sV0 + s * C::kKVBytes, C::kChunk, 1024);
-        const uint64_t pd = sw128_desc(sP0 + w * C::kPBytes, 16, 1024);
         const uint32_t od = tmem + C::kColO + w * D;
         const uint32_t acc0 = j >= 2 ? 1u : 0u;
+        if constexpr (C::kPTmem) {
+          // P_w: 128 lanes x 128 keys, two keys per column; 16 keys per step.
+          const uint32_t pt = tmem + C::kColP + w * 64;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          if (kk < nb * 4) {
-            const uint32_t poff = ((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4;
-            umma_ss(od, pd + poff, vd + kk * (2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kk < nb * 4) umma_ts(od, pt + kk * 8, vd + kk * (2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          }
+        } else {
+          const uint64_t pd = sw128_desc(sP0 + w * C::kPBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kk < nb * 4) {
+              const uint32_t poff = ((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4;
+              umma_ss(od, pd + poff, vd + kk * (2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+            }
           }
         }
         umma_commit(smem_u32(&bar_pfree[w]));
@@ -288,6 +304,7 @@ __global__ void __launch_bounds__(384, 1)
     // Row `row` of this warpgroup's P tile (keys 0-63 in the first 16 KB
     // chunk, keys 64-127 in the second), K-major with the 128-byte swizzle.
     const uint32_t prow = sP0 + w * C::kPBytes + (row >> 3) * 1024 + (row & 7) * 128;
+    const uint32_t pbuf = tmem + lane_off + C::kColP + w * 64;  // P_w in TMEM (d = 64)
     const float sl2 = a.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     const int kb_last = a.Kb - 1;
@@ -337,12 +354,15 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+      float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-      for (int c = 6; c < 126; c += 4) {
+      for (int c = 12; c < 124; c += 8) {
         mx0 = fmax3(mx0, s[c], s[c + 1]);
         mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
       }
-      const float rmax = fmax3(mx0, mx1, fmaxf(s[126], s[127]));
+      const float rmax = fmax3(fmax3(mx0, mx1, s[124]), fmax3(mx2, mx3, s[125]), fmaxf(s[126], s[127]));
       const float m_new = fmaxf(m_run, rmax * sl2);
       const bool need = m_new > m_run + 8.0f;  // always true for the first pair
       const float m_use = need ? m_new : m_run;
@@ -395,19 +415,25 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_st();
         }
       }
+      if constexpr (C::kPTmem) {
+        tmem_st32(pbuf, pk);
+        if (nb == 2) tmem_st32(pbuf + 32, pk + 32);
+        tmem_wait_st();
+      } else {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h == 1 && nb != 2) break;
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && nb != 2) break;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint32_t addr = prow + h * C::kChunk + ((g ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                       "r"(pk[h * 32 + g * 4]), "r"(pk[h * 32 + g * 4 + 1]),
-                       "r"(pk[h * 32 + g * 4 + 2]), "r"(pk[h * 32 + g * 4 + 3])
-                       : "memory");
+          for (int g = 0; g < 8; ++g) {
+            const uint32_t addr = prow + h * C::kChunk + ((g ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "r"(pk[h * 32 + g * 4]), "r"(pk[h * 32 + g * 4 + 1]),
+                         "r"(pk[h * 32 + g * 4 + 2]), "r"(pk[h * 32 + g * 4 + 3])
+                         : "memory");
+          }
         }
+        fence_proxy_async_smem();  // make P visible to the tensor core's async proxy
       }
-      fence_proxy_async_smem();  // make P visible to the tensor core's async proxy
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_pfull[w]));
       m_run = m_use;
