@@ -87,7 +87,7 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
   // The status word must start at zero; everything else is overwritten.
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
       (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
-      (e = launch_select(w.qbar, w.kbar, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
+      (e = launch_select(w.qbar, w.kbar, w.scores, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
                          w.cnt, st)) != cudaSuccess)
     return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   const char* why = nullptr;

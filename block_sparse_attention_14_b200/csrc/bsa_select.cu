@@ -102,8 +102,84 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ------------------------------------------------------------ block scores
-constexpr int kSelG = 16;          // query blocks per CTA (one warp each)
-constexpr int kSelThreads = 512;
+// S[bh][i][j] = Qbar_i . Kbar_j for every query block i and key block j, fp32
+// fmaf in ascending d order, rows padded to Kp = Kb rounded up to 4.  A
+// register-tiled fp32 GEMM: CTA tile 64 query blocks x 256 key blocks, 256
+// threads, 8 x 8 outputs per thread; Qbar of the tile is kept transposed in
+// shared memory and Kbar passes through in 32-wide d chunks (transposed, rows
+// padded to 260 floats), so each d step costs 4 shared loads per 64 FMAs.
+constexpr int kDotQ = 64, kDotK = 256, kDotDc = 32, kDotThreads = 256;
+constexpr int kDotKs = kDotK + 4;  // padded row of the transposed K chunk
+
+template <int D>
+constexpr size_t dots_smem() {
+  return sizeof(float) * (static_cast<size_t>(D) * kDotQ + static_cast<size_t>(kDotDc) * kDotKs);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __restrict__ qbar,
+                                                           const float* __restrict__ kbar, int Qb,
+                                                           int Kb, int Kp, float* __restrict__ S) {
+  extern __shared__ __align__(16) float dsm[];
+  float* Qs = dsm;                       // [D][kDotQ]
+  float* Ks = dsm + D * kDotQ;           // [kDotDc][kDotKs]
+  const int bh = blockIdx.z;
+  const int i0 = blockIdx.y * kDotQ;
+  const int j0 = blockIdx.x * kDotK;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 5;  // query blocks i0 + 8 ty ... + 7 (warp-uniform)
+  const int tx = tid & 31;  // key blocks j0 + 4 tx ... + 3 and j0 + 128 + 4 tx ... + 3
+  for (int e = tid; e < kDotQ * (D / 4); e += kDotThreads) {
+    const int q = e % kDotQ, d4 = e / kDotQ;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i0 + q < Qb) v = __ldg(reinterpret_cast<const float4*>(qbar + (static_cast<size_t>(bh) * Qb + i0 + q) * D) + d4);
+    Qs[(4 * d4 + 0) * kDotQ + q] = v.x;
+    Qs[(4 * d4 + 1) * kDotQ + q] = v.y;
+    Qs[(4 * d4 + 2) * kDotQ + q] = v.z;
+    Qs[(4 * d4 + 3) * kDotQ + q] = v.w;
+  }
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  for (int dc = 0; dc < D; dc += kDotDc) {
+    __syncthreads();  // the previous chunk is consumed (and Qs is written)
+    for (int e = tid; e < kDotK * (kDotDc / 4); e += kDotThreads) {
+      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + k < Kb)
+        v = __ldg(reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j0 + k) * D + dc) + c4);
+      Ks[(4 * c4 + 0) * kDotKs + k] = v.x;
+      Ks[(4 * c4 + 1) * kDotKs + k] = v.y;
+      Ks[(4 * c4 + 2) * kDotKs + k] = v.z;
+      Ks[(4 * c4 + 3) * kDotKs + k] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int dd = 0; dd < kDotDc; ++dd) {
+      const float4 qa = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty);
+      const float4 qb = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty + 4);
+      const float4 ka = *reinterpret_cast<const float4*>(Ks + dd * kDotKs + 4 * tx);
+      const float4 kb = *reinterpret_cast<const float4*>(Ks + dd * kDotKs + 128 + 4 * tx);
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + 8 * ty + a;
+    if (i >= Qb) break;
+    float* out = S + (static_cast<size_t>(bh) * Qb + i) * Kp;
+    const int ja = j0 + 4 * tx, jb = j0 + 128 + 4 * tx;
+    if (ja < Kp) *reinterpret_cast<float4*>(out + ja) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    if (jb < Kp) *reinterpret_cast<float4*>(out + jb) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+  }
+}
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
 // +0 and -0 map to the same key.
@@ -112,56 +188,48 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Dot products Qbar_i . Kbar_j for kSelG query blocks and every key block,
-// accumulated in fp32 in ascending d order, into sc[g][j].
-template <int D>
-__device__ __forceinline__ void block_dots(const float* __restrict__ qbar,
-                                           const float* __restrict__ kbar, int bh, int i0,
-                                           int Qb, int Kb, float* sq, float* sc) {
-  for (int e = threadIdx.x; e < kSelG * D; e += kSelThreads) {
-    const int g = e / D;
-    const int i = i0 + g;
-    sq[e] = (i < Qb) ? qbar[(static_cast<size_t>(bh) * Qb + i) * D + (e % D)] : 0.f;
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < Kb; j += kSelThreads) {
-    const float4* kr = reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j) * D);
-    float acc[kSelG];
-#pragma unroll
-    for (int g = 0; g < kSelG; ++g) acc[g] = 0.f;
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = __ldg(kr + d4);
-#pragma unroll
-      for (int g = 0; g < kSelG; ++g) {
-        const float4 qv = reinterpret_cast<const float4*>(sq + g * D)[d4];
-        acc[g] = fmaf(qv.x, kv.x, acc[g]);
-        acc[g] = fmaf(qv.y, kv.y, acc[g]);
-        acc[g] = fmaf(qv.z, kv.z, acc[g]);
-        acc[g] = fmaf(qv.w, kv.w, acc[g]);
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < kSelG; ++g) sc[g * Kb + j] = acc[g];
-  }
-  __syncthreads();
+// The row kernels below run one warp per (bh, i) row, eight rows per CTA; the
+// warp first copies its score row into shared memory.
+constexpr int kRowWarps = 8;
+
+__device__ __forceinline__ float* stage_row(const float* __restrict__ S, size_t row, int Kp,
+                                            float* dst) {
+  const int lane = threadIdx.x & 31;
+  const float4* src = reinterpret_cast<const float4*>(S + row * Kp);
+  for (int j4 = lane; j4 < Kp / 4; j4 += 32) reinterpret_cast<float4*>(dst)[j4] = src[j4];
+  __syncwarp();
+  return dst;
 }
 
 // Top-k of one row of dot products by one warp: a most-significant-digit radix
 // select over the float keys finds the kk-th largest key T and how many of the
 // keys equal to T are kept; the row is then emitted in ascending block order
-// (keys above T, plus the first `need_eq` keys equal to T).
+// (keys above T, plus the first `need_eq` keys equal to T).  The digits are
+// taken of (key - kmin) from the top bit of the row's key range down, so the
+// first histogram spreads over all 256 buckets instead of the few that the
+// top byte of similar floats falls in (which serialised the shared atomics).
 __device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, uint8_t* mask_row,
                               int16_t* idx_row, int32_t* cnt_out) {
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, pmask = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j = lane; j < Kb; j += 32) {
+    const uint32_t u = float_key(row[j]);
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  const int nbits = 32 - __clz(static_cast<int>(kmax - kmin));  // bits of the range (0 if flat)
+  uint32_t prefix = 0, pmask = 0;  // over v = key - kmin
   int remaining = kk;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int hi = nbits; hi > 0;) {
+    const int lo = hi > 8 ? hi - 8 : 0;
+    const uint32_t dmask = (1u << (hi - lo)) - 1u;
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
     for (int j = lane; j < Kb; j += 32) {
-      const uint32_t u = float_key(row[j]);
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      const uint32_t v = float_key(row[j]) - kmin;
+      if ((v & pmask) == prefix) atomicAdd(&hist[(v >> lo) & dmask], 1u);
     }
     __syncwarp();
     // Lane l owns buckets 255-8l ... 248-8l (descending).
@@ -196,11 +264,12 @@ __device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, 
     bucket = __shfl_sync(0xffffffffu, bucket, src);
     above = __shfl_sync(0xffffffffu, above, src);
     remaining -= static_cast<int>(above);
-    prefix |= bucket << shift;
-    pmask |= 255u << shift;
+    prefix |= bucket << lo;
+    pmask |= dmask << lo;
+    hi = lo;
     __syncwarp();
   }
-  const uint32_t T = prefix;
+  const uint32_t T = prefix + kmin;
   const int need_eq = remaining;  // keys equal to T still to keep, lowest index first
   int eq_seen = 0, kept = 0;
   const unsigned lt = (1u << lane) - 1u;
@@ -326,26 +395,19 @@ __device__ void warp_cdf_row(float* row, int Kb, float scale, float tau, uint8_t
   if (lane == 0) *cnt_out = kept;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSelThreads) select_cdf_kernel(const float* __restrict__ qbar,
-                                                                 const float* __restrict__ kbar,
-                                                                 int Qb, int Kb, float scale,
-                                                                 float tau,
-                                                                 uint8_t* __restrict__ mask_out,
-                                                                 int16_t* __restrict__ idx,
-                                                                 int32_t* __restrict__ cnt) {
+__global__ void __launch_bounds__(32 * kRowWarps) select_cdf_kernel(const float* __restrict__ S,
+                                                                   int rows, int Kb, int Kp,
+                                                                   float scale, float tau,
+                                                                   uint8_t* __restrict__ mask_out,
+                                                                   int16_t* __restrict__ idx,
+                                                                   int32_t* __restrict__ cnt) {
   extern __shared__ __align__(16) float smem[];
-  float* sq = smem;
-  float* sc = sq + kSelG * D;
-  const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kSelG;
-  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
   const int w = threadIdx.x >> 5;
-  const int i = i0 + w;
-  if (i >= Qb) return;
-  const size_t row = static_cast<size_t>(bh) * Qb + i;
-  warp_cdf_row(sc + w * Kb, Kb, scale, tau, mask_out ? mask_out + row * Kb : nullptr,
-               idx + row * Kb, cnt + row);
+  const size_t row = static_cast<size_t>(blockIdx.x) * kRowWarps + w;
+  if (row >= static_cast<size_t>(rows)) return;
+  float* r = stage_row(S, row, Kp, smem + w * Kp);
+  warp_cdf_row(r, Kb, scale, tau, mask_out ? mask_out + row * Kb : nullptr, idx + row * Kb,
+               cnt + row);
 }
 
 // Kept count for a fraction of E blocks: clamp(ceil(topk * E), 1, E) in double
@@ -356,50 +418,38 @@ __device__ __forceinline__ int keep_count_dev(float topk, int E) {
   return max(1, min(E, k));
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ qbar,
-                                                             const float* __restrict__ kbar,
-                                                             int Qb, int Kb, int kk, float topk,
-                                                             int causal,
-                                                             uint8_t* __restrict__ mask_out,
-                                                             int16_t* __restrict__ idx,
-                                                             int32_t* __restrict__ cnt) {
-  extern __shared__ __align__(16) float smem[];
-  float* sq = smem;                              // [kSelG][D]
-  float* sc = sq + kSelG * D;                    // [kSelG][Kb]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sc + kSelG * Kb);  // [16][256]
-  const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kSelG;
-  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
+__global__ void __launch_bounds__(32 * kRowWarps) select_kernel(const float* __restrict__ S, int rows,
+                                                               int Qb, int Kb, int Kp, int kk,
+                                                               float topk, int causal,
+                                                               uint8_t* __restrict__ mask_out,
+                                                               int16_t* __restrict__ idx,
+                                                               int32_t* __restrict__ cnt) {
+  extern __shared__ __align__(16) float smem[];  // [kRowWarps][Kp] rows, [kRowWarps][256] hist
   const int w = threadIdx.x >> 5;
-  const int i = i0 + w;
-  if (i >= Qb) return;
-  const size_t row = static_cast<size_t>(bh) * Qb + i;
+  const size_t row = static_cast<size_t>(blockIdx.x) * kRowWarps + w;
+  if (row >= static_cast<size_t>(rows)) return;
+  float* r = stage_row(S, row, Kp, smem + w * Kp);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + kRowWarps * Kp) + w * 256;
+  const int i = static_cast<int>(row % static_cast<size_t>(Qb));
   // Causal: query block i may use key blocks 0 .. 2i+1 only; top-k runs over those.
   const int Ke = causal ? min(2 * i + 2, Kb) : Kb;
   const int k_row = causal ? keep_count_dev(topk, Ke) : kk;
   uint8_t* mrow = mask_out ? mask_out + row * Kb : nullptr;
-  warp_topk_row(sc + w * Kb, Ke, k_row, hist + w * 256, mrow, idx + row * Kb, cnt + row);
+  warp_topk_row(r, Ke, k_row, hist, mrow, idx + row * Kb, cnt + row);
   if (mrow != nullptr)
     for (int j = Ke + (threadIdx.x & 31); j < Kb; j += 32) mrow[j] = 0;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSelThreads) block_scores_kernel(const float* __restrict__ qbar,
-                                                                   const float* __restrict__ kbar,
-                                                                   int Qb, int Kb, float scale,
-                                                                   float* __restrict__ p_out) {
+__global__ void __launch_bounds__(32 * kRowWarps) block_scores_kernel(const float* __restrict__ S,
+                                                                     int rows, int Kb, int Kp,
+                                                                     float scale,
+                                                                     float* __restrict__ p_out) {
   extern __shared__ __align__(16) float smem[];
-  float* sq = smem;
-  float* sc = sq + kSelG * D;
-  const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * kSelG;
-  block_dots<D>(qbar, kbar, bh, i0, Qb, Kb, sq, sc);
   const int w = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int i = i0 + w;
-  if (i >= Qb) return;
-  const float* r = sc + w * Kb;
+  const size_t row = static_cast<size_t>(blockIdx.x) * kRowWarps + w;
+  if (row >= static_cast<size_t>(rows)) return;
+  const float* r = stage_row(S, row, Kp, smem + w * Kp);
   float mx = -INFINITY;
   for (int j = lane; j < Kb; j += 32) mx = fmaxf(mx, r[j]);
 #pragma unroll
@@ -409,7 +459,7 @@ __global__ void __launch_bounds__(kSelThreads) block_scores_kernel(const float* 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float inv = 1.f / sum;
-  float* out = p_out + (static_cast<size_t>(bh) * Qb + i) * Kb;
+  float* out = p_out + row * Kb;
   for (int j = lane; j < Kb; j += 32) out[j] = expf((r[j] - mx) * scale) * inv;
 }
 
@@ -438,9 +488,28 @@ __global__ void __launch_bounds__(256) compact_kernel(const uint8_t* __restrict_
   if (lane == 0) cnt[row] = kept;
 }
 
-size_t select_smem(int d, int Kb, bool with_hist) {
-  return sizeof(float) * (static_cast<size_t>(kSelG) * d + static_cast<size_t>(kSelG) * Kb) +
-         (with_hist ? sizeof(uint32_t) * 16 * 256 : 0);
+size_t row_smem(int Kp, bool with_hist) {
+  return sizeof(float) * kRowWarps * static_cast<size_t>(Kp) +
+         (with_hist ? sizeof(uint32_t) * kRowWarps * 256 : 0);
+}
+
+cudaError_t launch_dots(const float* qbar, const float* kbar, int BH, int Qb, int Kb, int d,
+                        float* S, cudaStream_t st) {
+  const int Kp = padded_kb(Kb);
+  dim3 grid((Kb + kDotK - 1) / kDotK, (Qb + kDotQ - 1) / kDotQ, BH);
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(dots_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(dots_smem<128>()));
+    if (e != cudaSuccess) return e;
+    dots_kernel<128><<<grid, kDotThreads, dots_smem<128>(), st>>>(qbar, kbar, Qb, Kb, Kp, S);
+  } else {
+    e = cudaFuncSetAttribute(dots_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(dots_smem<64>()));
+    if (e != cudaSuccess) return e;
+    dots_kernel<64><<<grid, kDotThreads, dots_smem<64>(), st>>>(qbar, kbar, Qb, Kb, Kp, S);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -461,74 +530,58 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* qbar, const float* kbar, int BH, int N, int d, int kk,
-                          float topk, int causal, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
-                          cudaStream_t st) {
+cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int BH, int N, int d,
+                          int kk, float topk, int causal, uint8_t* mask_out, int16_t* idx,
+                          int32_t* cnt, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
-  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
-  const size_t smem = select_smem(d, Kb, true);
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    select_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, topk, causal, mask_out,
-                                                        idx, cnt);
-  } else {
-    e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    select_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, kk, topk, causal, mask_out,
-                                                       idx, cnt);
-  }
+  const int Kp = padded_kb(Kb);
+  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
+  if (e != cudaSuccess) return e;
+  const int rows = BH * Qb;
+  const size_t smem = row_smem(Kp, true);
+  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  select_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+      scores, rows, Qb, Kb, Kp, kk, topk, causal, mask_out, idx, cnt);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select_cdf(const float* qbar, const float* kbar, int BH, int N, int d,
-                              float threshold, uint8_t* mask_out, int16_t* idx, int32_t* cnt,
-                              cudaStream_t st) {
+cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int BH, int N,
+                              int d, float threshold, uint8_t* mask_out, int16_t* idx,
+                              int32_t* cnt, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
-  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
-  const size_t smem = select_smem(d, Kb, false);
+  const int Kp = padded_kb(Kb);
+  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
+  if (e != cudaSuccess) return e;
+  const int rows = BH * Qb;
+  const size_t smem = row_smem(Kp, false);
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(select_cdf_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    select_cdf_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, threshold,
-                                                            mask_out, idx, cnt);
-  } else {
-    e = cudaFuncSetAttribute(select_cdf_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    select_cdf_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, threshold,
-                                                           mask_out, idx, cnt);
-  }
+  e = cudaFuncSetAttribute(select_cdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  select_cdf_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+      scores, rows, Kb, Kp, scale, threshold, mask_out, idx, cnt);
   return cudaGetLastError();
 }
 
-cudaError_t launch_block_scores(const float* qbar, const float* kbar, int BH, int N, int d,
-                                float* p_out, cudaStream_t st) {
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int BH, int N,
+                                int d, float* p_out, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
-  dim3 grid((Qb + kSelG - 1) / kSelG, BH);
-  const size_t smem = select_smem(d, Kb, false);
+  const int Kp = padded_kb(Kb);
+  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
+  if (e != cudaSuccess) return e;
+  const int rows = BH * Qb;
+  const size_t smem = row_smem(Kp, false);
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(block_scores_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    block_scores_kernel<128><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, p_out);
-  } else {
-    e = cudaFuncSetAttribute(block_scores_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    block_scores_kernel<64><<<grid, kSelThreads, smem, st>>>(qbar, kbar, Qb, Kb, scale, p_out);
-  }
+  e = cudaFuncSetAttribute(block_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  block_scores_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+      scores, rows, Kb, Kp, scale, p_out);
   return cudaGetLastError();
 }
 

@@ -72,7 +72,8 @@ const char* bsa_status_string(bsa_status s);
  * (static, thread-local string; empty if none). */
 const char* bsa_last_error_message(void);
 
-/* Workspace bytes needed for a shape: pooled means, the compacted per-query-
+/* Workspace bytes needed for a shape: pooled means, the fp32 block-score
+ * matrix (B*H*Qb rows of Kb rounded up to 4 floats), the compacted per-query-
  * block key-block index list, its counts and the device status word.  Returns 0
  * for a shape the library rejects. */
 size_t bsa_workspace_bytes(bsa_shape s);

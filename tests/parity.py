@@ -79,3 +79,16 @@ def compare_cdf_masks(mask_gpu: torch.Tensor, mask_ref: np.ndarray, P_ref: np.nd
     diff = np.any(mg != mask_ref, axis=-1)
     ex = O.cdf_exempt_rows(P_ref, tau)
     return int((diff & ~ex).sum()), int(ex.sum())
+
+
+def workspace_lists(ws: torch.Tensor, BH: int, Qb: int, Kb: int, d: int):
+    """The compacted (idx, cnt) lists from a workspace, at the offsets of the
+    layout include/bsa.h documents: status 256 | qbar | kbar | block scores (rows
+    padded to 4 floats) | idx int16 | cnt int32, each rounded up to 256 bytes."""
+    r = lambda x: (x + 255) // 256 * 256
+    Kp = (Kb + 3) // 4 * 4
+    o_idx = 256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4) + r(BH * Qb * Kp * 4)
+    o_cnt = o_idx + r(BH * Qb * Kb * 2)
+    idx = ws[o_idx:o_idx + BH * Qb * Kb * 2].view(torch.int16).view(BH * Qb, Kb).cpu().numpy()
+    cnt = ws[o_cnt:o_cnt + BH * Qb * 4].view(torch.int32).cpu().numpy()
+    return idx, cnt

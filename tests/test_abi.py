@@ -34,12 +34,15 @@ def test_status_strings():
 
 
 def test_workspace_bytes():
-    # status 256 + qbar + kbar + idx (int16) + cnt, each rounded up to 256 bytes
+    # status 256 + qbar + kbar + block scores (fp32, rows padded to 4) + idx (int16)
+    # + cnt, each rounded up to 256 bytes
     def r(x):
         return (x + 255) // 256 * 256
     for B, H, N, d in [(1, 40, 75600, 128), (2, 30, 17776, 64), (1, 1, 1, 64), (1, 2, 1024, 64)]:
         BH, Qb, Kb = B * H, -(-N // 128), -(-N // 64)
-        want = 256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4) + r(BH * Qb * Kb * 2) + r(BH * Qb * 4)
+        Kp = (Kb + 3) // 4 * 4
+        want = (256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4) + r(BH * Qb * Kp * 4)
+                + r(BH * Qb * Kb * 2) + r(BH * Qb * 4))
         assert bsa.workspace_bytes(B, H, N, d) == want
     for bad in [(0, 1, 64, 64), (1, 1, 64, 96), (1, 1, 131073, 64), (1, 1, 0, 128), (256, 256, 64, 64)]:
         assert bsa.workspace_bytes(*bad) == 0

@@ -14,6 +14,7 @@ import block_sparse_attention_14_b200 as bsa
 from block_sparse_attention_14_b200 import workloads as W
 from oracle import bsa_oracle as O
 from tests.parity import assert_close, compare_masks, sampled_blocks
+from tests import parity as P
 
 pytestmark = pytest.mark.gpu
 
@@ -88,11 +89,7 @@ def test_wan14b_caller_mask(density):
     bsa.last_device_status(ws)
     # The caller mask passes bit-exactly into the kept-block lists.
     BH, Qb, Kb = wl.B * wl.H, wl.Qb, wl.Kb
-    r = lambda x: (x + 255) // 256 * 256
-    o_idx = 256 + r(BH * Qb * wl.d * 4) + r(BH * Kb * wl.d * 4)
-    o_cnt = o_idx + r(BH * Qb * Kb * 2)
-    idx = ws[o_idx:o_idx + BH * Qb * Kb * 2].view(torch.int16).view(BH * Qb, Kb).cpu().numpy()
-    cnt = ws[o_cnt:o_cnt + BH * Qb * 4].view(torch.int32).cpu().numpy()
+    idx, cnt = P.workspace_lists(ws, BH, Qb, Kb, wl.d)
     m = mask.view(BH * Qb, Kb).numpy()
     assert np.array_equal(cnt, m.sum(1))
     order = np.argsort(m == 0, axis=1, kind="stable")

@@ -10,6 +10,7 @@ import block_sparse_attention_14_b200 as bsa
 from block_sparse_attention_14_b200 import workloads as W
 from oracle import bsa_oracle as O
 from tests.parity import assert_close, compare_masks
+from tests import parity as P
 
 pytestmark = pytest.mark.gpu
 
@@ -128,12 +129,8 @@ def test_compaction_is_exact(cuda_device):
     ws = bsa.make_workspace(B, H, N, d)
     bsa.block_sparse_attn_fwd(q, k, v, mask.cuda(), workspace=ws)
     torch.cuda.synchronize()
-    r = lambda x: (x + 255) // 256 * 256
     BH = B * H
-    o_idx = 256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4)
-    o_cnt = o_idx + r(BH * Qb * Kb * 2)
-    idx = ws[o_idx:o_idx + BH * Qb * Kb * 2].view(torch.int16).view(BH * Qb, Kb).cpu().numpy()
-    cnt = ws[o_cnt:o_cnt + BH * Qb * 4].view(torch.int32).cpu().numpy()
+    idx, cnt = P.workspace_lists(ws, BH, Qb, Kb, d)
     m = mask.view(BH * Qb, Kb).numpy()
     for row in range(BH * Qb):
         want = np.flatnonzero(m[row])
