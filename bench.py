@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import glob
 import hashlib
 import io
 import json
@@ -47,7 +48,7 @@ METRIC = "ms/call and dense-equiv TFLOPS, Wan-14B-shaped topk=0.5, % of bf16 TC 
 UNIT = "dense-equiv TFLOPS"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_14_b200", "csrc", "bsa_attn.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_fwd_kernel_wan14b_ncu.md")
+TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "bsa_fwd_kernel_*_ncu.md")
 
 
 def parse_args():
@@ -81,17 +82,17 @@ def attn_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """Per-launch DRAM bytes of the attention kernel from a committed ncu summary,
-    valid only if it was taken on the current kernel source."""
-    if not os.path.exists(TRAFFIC_FILE):
-        return None
+    """Per-launch DRAM bytes of the attention kernel from a committed ncu summary
+    (profiles/bsa_fwd_kernel_*_ncu.md), valid only if it was taken on the current
+    kernel source."""
     want = attn_source_hash()
-    with open(TRAFFIC_FILE) as f:
-        for line in f:
-            if line.startswith("traffic_bytes_per_launch:"):
-                parts = dict(x.split("=", 1) for x in line.split(":", 1)[1].split() if "=" in x)
-                if parts.get("workload") == workload and parts.get("source") == want:
-                    return float(parts["bytes"])
+    for path in sorted(glob.glob(TRAFFIC_GLOB)):
+        with open(path) as f:
+            for line in f:
+                if line.startswith("traffic_bytes_per_launch:"):
+                    parts = dict(x.split("=", 1) for x in line.split(":", 1)[1].split() if "=" in x)
+                    if parts.get("workload") == workload and parts.get("source") == want:
+                        return float(parts["bytes"])
     return None
 
 
@@ -360,7 +361,7 @@ def run_b200(args, world, rank, local):
                 "peak_kind": f"bf16 dense burst, of {kind}",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "algorithmic_flops_per_launch": kept_flops, "avg_launch_ms": attn_s * 1e3}
-    roofline_select = {"bound": "hbm", "kernel": "pool_kernel + select_kernel",
+    roofline_select = {"bound": "hbm", "kernel": "pool_kernel + dots_kernel + select_kernel",
                        "achieved": sel_bytes / sel_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": sel_bytes / sel_s / 1e9 / peaks["hbm_gbs"],
                        "algorithmic_bytes_per_call": sel_bytes, "avg_call_ms": sel_s * 1e3}
@@ -378,7 +379,7 @@ def run_b200(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(wl, args.topk, H),
             "roofline": roofline, "roofline_select": roofline_select, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 3 * K, "clocks": clk,
+            "gpu_launches": 4 * K, "clocks": clk,  # pool, dots, select, attention
             "breakdown": {"select_ms": sel_s * 1e3, "attention_ms": attn_s * 1e3,
                           "fused_call_ms": fused_ms, "density": density,
                           "kept_tflop": kept_flops / 1e12, "dense_tflop": dense_flops / 1e12},
