@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_select_cdf.argtypes = [vp, vp, Shape, f32, vp, vp, sz, vp]
         L.sparse_attn_cdf.restype = i32
         L.sparse_attn_cdf.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp, sz, vp]
+        L.sparse_attn_topk_host.restype = i32
+        L.sparse_attn_topk_host.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp, vp, vp, vp, sz, i32, vp]
         L.block_sparse_attn_plan.restype = i32
         L.block_sparse_attn_plan.argtypes = [vp, Shape, i32, vp, sz, vp]
         L.block_sparse_attn_apply.restype = i32
@@ -194,6 +196,34 @@ def sparse_attn_topk(q, k, v, topk: float = 0.5, is_causal: bool = False, *, out
                                   int(bool(is_causal)), out.data_ptr(),
                                   mask.data_ptr() if mask is not None else None, wp, wn, _stream(q)))
     return (out, mask) if return_mask else out
+
+
+def sparse_attn_topk_host(q_host, k_host, v_host, topk: float = 0.5, is_causal: bool = False, *,
+                          out_host=None, device_buffers=None, workspace=None, chunks: int = 0,
+                          device="cuda"):
+    """sparse_attn_topk on pinned host tensors, with the host<->device copies
+    pipelined over chunks of heads.  device_buffers: (q, k, v, out) device tensors
+    of the same shape (allocated if None).  Runs on the current stream of
+    `device`; returns out_host once that stream has finished."""
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_pinned():
+            raise ValueError(f"{name} must be a contiguous pinned bf16 host tensor")
+        if t.shape != q_host.shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(q_host.shape)}")
+    if out_host is None:
+        out_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
+    if device_buffers is None:
+        device_buffers = tuple(torch.empty(q_host.shape, dtype=torch.bfloat16, device=device) for _ in range(4))
+    qd, kd, vd, od = device_buffers
+    _qkv(qd, kd, vd)
+    _qkv(qd, od)
+    ws, wp, wn = _ws(qd, workspace)
+    _check(lib().sparse_attn_topk_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                       _shape_of(qd), float(topk), int(bool(is_causal)),
+                                       out_host.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
+                                       od.data_ptr(), wp, wn, int(chunks), _stream(qd)))
+    torch.cuda.current_stream(qd.device).synchronize()
+    return out_host
 
 
 def block_sparse_attn_fwd(q, k, v, mask_id=None, is_causal: bool = False, *, out=None, workspace=None):

@@ -89,6 +89,36 @@ int keep_count(float topk, int Kb) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+bsa_status check_pinned(const void* p, const char* name) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the error state the failed query left
+    return fail(BSA_ERR_INVALID_ARG, "%s: pointer attributes unavailable", name);
+  }
+  if (a.type != cudaMemoryTypeHost)
+    return fail(BSA_ERR_INVALID_ARG,
+                "%s must be page-locked host memory (cudaHostAlloc or cudaHostRegister)", name);
+  return BSA_OK;
+}
+
+// Streams and events of one host-pipelined call.  Destroying them while work
+// is still pending is allowed: CUDA releases them once that work completes.
+struct PipelineResources {
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t events[2 + 2 * 64] = {};
+  int n_events = 0;
+  cudaError_t event(cudaEvent_t* e) {
+    cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+    if (r == cudaSuccess) events[n_events++] = *e;
+    return r;
+  }
+  ~PipelineResources() {
+    for (int i = 0; i < n_events; ++i) cudaEventDestroy(events[i]);
+    if (copy_in) cudaStreamDestroy(copy_in);
+    if (copy_out) cudaStreamDestroy(copy_out);
+  }
+};
+
 }  // namespace
 
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
@@ -279,6 +309,110 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
                                    g_timeout_ns.load(), st, &why);
   if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
   return BSA_OK;
+}
+
+bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const void* v_host,
+                                 bsa_shape s, float topk, int is_causal, void* out_host, void* q_dev,
+                                 void* k_dev, void* v_dev, void* out_dev, void* ws, size_t ws_bytes,
+                                 int chunks, void* stream) {
+  g_last_error[0] = 0;
+  BSA_TRY(check_shape(s));
+  BSA_TRY(check_tensor(q_host, "q_host"));
+  BSA_TRY(check_tensor(k_host, "k_host"));
+  BSA_TRY(check_tensor(v_host, "v_host"));
+  BSA_TRY(check_tensor(out_host, "out_host"));
+  BSA_TRY(check_tensor(q_dev, "q_dev"));
+  BSA_TRY(check_tensor(k_dev, "k_dev"));
+  BSA_TRY(check_tensor(v_dev, "v_dev"));
+  BSA_TRY(check_tensor(out_dev, "out_dev"));
+  BSA_TRY(check_topk(topk));
+  Workspace w;
+  BSA_TRY(check_ws(s, ws, ws_bytes, &w));
+  BSA_TRY(check_pinned(q_host, "q_host"));
+  BSA_TRY(check_pinned(k_host, "k_host"));
+  BSA_TRY(check_pinned(v_host, "v_host"));
+  BSA_TRY(check_pinned(out_host, "out_host"));
+  const int BH = s.B * s.H;
+  const int Qb = (s.N + kBlockQ - 1) / kBlockQ;
+  const int max_chunks = BH < 64 ? BH : 64;
+  int nc = chunks;
+  if (nc <= 0) {
+    // About eight waves of attention CTAs (one per SM) per chunk: enough to keep
+    // the tail of each chunk small, small enough to keep the pipeline's fill
+    // and drain (one chunk's copy in and copy out) short.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+    const int64_t ctas = static_cast<int64_t>(BH) * Qb;
+    nc = static_cast<int>((ctas + 4 * sms) / (8 * sms));
+  }
+  nc = nc < 1 ? 1 : (nc > max_chunks ? max_chunks : nc);
+  const int Kb = (s.N + kBlockK - 1) / kBlockK;
+  const int kk = keep_count(topk, Kb);
+  const size_t head_bytes = static_cast<size_t>(s.N) * s.d * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  PipelineResources r;
+  cudaEvent_t e_start = nullptr, e_end = nullptr;
+  BSA_CUDA(cudaStreamCreateWithFlags(&r.copy_in, cudaStreamNonBlocking), "copy stream");
+  BSA_CUDA(cudaStreamCreateWithFlags(&r.copy_out, cudaStreamNonBlocking), "copy stream");
+  BSA_CUDA(r.event(&e_start), "event");
+  BSA_CUDA(r.event(&e_end), "event");
+  // Nothing of this call starts before the work already queued on `stream`.
+  BSA_CUDA(cudaEventRecord(e_start, st), "event record");
+  BSA_CUDA(cudaStreamWaitEvent(r.copy_in, e_start, 0), "stream wait");
+  BSA_CUDA(cudaStreamWaitEvent(r.copy_out, e_start, 0), "stream wait");
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+
+  // Chunk c: heads [h0, h1) of the flattened B*H; copy in on copy_in, compute on
+  // `stream` with the chunk's own workspace layout (status word at offset 0 in
+  // every layout), copy out on copy_out.  Chunks are disjoint byte ranges.
+  const auto run = [&]() -> bsa_status {
+    const char* qh = static_cast<const char*>(q_host);
+    const char* kh = static_cast<const char*>(k_host);
+    const char* vh = static_cast<const char*>(v_host);
+    char* oh = static_cast<char*>(out_host);
+    char* qd = static_cast<char*>(q_dev);
+    char* kd = static_cast<char*>(k_dev);
+    char* vd = static_cast<char*>(v_dev);
+    char* od = static_cast<char*>(out_dev);
+    for (int c = 0; c < nc; ++c) {
+      const int h0 = static_cast<int>(static_cast<int64_t>(BH) * c / nc);
+      const int h1 = static_cast<int>(static_cast<int64_t>(BH) * (c + 1) / nc);
+      const int bhc = h1 - h0;
+      if (bhc == 0) continue;
+      const size_t off = static_cast<size_t>(h0) * head_bytes;
+      const size_t bytes = static_cast<size_t>(bhc) * head_bytes;
+      cudaEvent_t e_in = nullptr, e_done = nullptr;
+      BSA_CUDA(r.event(&e_in), "event");
+      BSA_CUDA(r.event(&e_done), "event");
+      BSA_CUDA(cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "q copy in");
+      BSA_CUDA(cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "k copy in");
+      BSA_CUDA(cudaMemcpyAsync(vd + off, vh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "v copy in");
+      BSA_CUDA(cudaEventRecord(e_in, r.copy_in), "event record");
+      BSA_CUDA(cudaStreamWaitEvent(st, e_in, 0), "stream wait");
+      Workspace wc;
+      workspace_layout(1, bhc, s.N, s.d, &wc, ws);
+      BSA_CUDA(launch_pool(qd + off, kd + off, bhc, s.N, s.d, wc.qbar, wc.kbar, st), "pool kernel launch");
+      BSA_CUDA(launch_select(wc.qbar, wc.kbar, wc.scores, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr,
+                             wc.idx, wc.cnt, st),
+               "select kernel launch");
+      const char* why = nullptr;
+      cudaError_t e = launch_attention(qd + off, kd + off, vd + off, od + off, bhc, s.N, s.d, is_causal != 0,
+                                       wc.idx, wc.cnt, wc.status, g_timeout_ns.load(), st, &why);
+      if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
+      BSA_CUDA(cudaEventRecord(e_done, st), "event record");
+      BSA_CUDA(cudaStreamWaitEvent(r.copy_out, e_done, 0), "stream wait");
+      BSA_CUDA(cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, r.copy_out), "out copy");
+    }
+    return BSA_OK;
+  };
+  const bsa_status status = run();
+  // `stream` waits for the last copy out, also after a failure part-way, so
+  // that synchronising it covers everything this call queued.
+  if (cudaEventRecord(e_end, r.copy_out) == cudaSuccess) cudaStreamWaitEvent(st, e_end, 0);
+  return status;
 }
 
 bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, int is_causal, void* ws,

@@ -171,6 +171,32 @@ bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
                                     float topk, int is_causal, void* out, uint8_t* mask_out,
                                     void* stream);
 
+/* sparse_attn_topk on HOST buffers, pipelined over chunks of heads: while the
+ * kernels of chunk c run on `stream`, chunk c+1's q/k/v are copied in on one
+ * internal copy stream and chunk c-1's output is copied out on another.  The
+ * pages have no counterpart: heads are independent (the same selection and
+ * attention run per head), so this only overlaps PCIe transfers with the
+ * compute of sparse_attn_topk, and out_host receives exactly the bytes that
+ * sparse_attn_topk writes.
+ *  - q_host, k_host, v_host (read), out_host (written): page-locked host memory
+ *    (cudaHostAlloc / cudaHostRegister; anything else is BSA_ERR_INVALID_ARG),
+ *    bf16 [B, H, N, d], 16-byte aligned.
+ *  - q_dev, k_dev, v_dev, out_dev: device buffers of the same size, owned by the
+ *    caller; the call overwrites all four.
+ *  - ws, ws_bytes: a workspace for the full shape (bsa_workspace_bytes(s)).
+ *  - chunks: number of head chunks, clamped to [1, min(B*H, 64)]; <= 0 picks
+ *    about eight waves of attention CTAs (one per SM) per chunk.
+ *  - stream: the compute stream.  Nothing starts before the work already queued
+ *    on it, and it waits for the last copy out, so synchronising `stream` (then
+ *    bsa_last_device_status) covers the whole call.  Non-causal and causal as in
+ *    sparse_attn_topk; no mask is written.  The call creates two streams and
+ *    their events and releases them when the work completes, so calls from
+ *    several host threads do not share state. */
+bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const void* v_host,
+                                 bsa_shape s, float topk, int is_causal, void* out_host, void* q_dev,
+                                 void* k_dev, void* v_dev, void* out_dev, void* ws, size_t ws_bytes,
+                                 int chunks, void* stream);
+
 /* Token reordering (after the AB-Attention README's "Optional cube layout" and
  * the Morton3D ordering of the LightX2V page "Sol-Attn on Wan2.1"): writes
  * perm_out (host int32, text + T*Hg*Wg entries), perm[new] = old, for a

@@ -90,6 +90,7 @@ def test_other_calls_reject_bad_arguments():
     assert L.sparse_attn_block_scores(256, 256, s, None, 512, n, None) == 1
     assert L.sparse_attn_block_scores(256, 256, bsa.Shape(1, 2, 300, 32), 1024, 512, n, None) == 1
     assert L.bsa_last_device_status(None, None) == 1
+    assert L.sparse_attn_topk_host(None, 256, 256, s, 0.5, 0, 256, 256, 256, 256, 256, 512, n, 0, None) == 1
 
 
 def test_keep_count_matches_oracle_reading():
