@@ -127,15 +127,16 @@ void set_last_error(const char* msg) {
   snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
 }
 
-size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base) {
+size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base, int score_heads) {
   const size_t BH = static_cast<size_t>(B) * H;
+  const size_t SH = (score_heads <= 0 || static_cast<size_t>(score_heads) > BH) ? BH : score_heads;
   const size_t Qb = (static_cast<size_t>(N) + kBlockQ - 1) / kBlockQ;
   const size_t Kb = (static_cast<size_t>(N) + kBlockK - 1) / kBlockK;
   size_t off = 0;
   const size_t o_status = off; off = align256(off + sizeof(DeviceStatus));
   const size_t o_qbar = off;   off = align256(off + BH * Qb * d * sizeof(float));
   const size_t o_kbar = off;   off = align256(off + BH * Kb * d * sizeof(float));
-  const size_t o_sc = off;     off = align256(off + BH * Qb * padded_kb(static_cast<int>(Kb)) * sizeof(float));
+  const size_t o_sc = off;     off = align256(off + SH * Qb * padded_kb(static_cast<int>(Kb)) * sizeof(float));
   const size_t o_idx = off;    off = align256(off + BH * Qb * Kb * sizeof(int16_t));
   const size_t o_cnt = off;    off = align256(off + BH * Qb * sizeof(int32_t));
   if (ws != nullptr) {
@@ -144,6 +145,7 @@ size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base) {
     ws->qbar = reinterpret_cast<float*>(b + o_qbar);
     ws->kbar = reinterpret_cast<float*>(b + o_kbar);
     ws->scores = reinterpret_cast<float*>(b + o_sc);
+    ws->score_heads = static_cast<int>(SH);
     ws->idx = reinterpret_cast<int16_t*>(b + o_idx);
     ws->cnt = reinterpret_cast<int32_t*>(b + o_cnt);
     ws->bytes = off;
@@ -192,7 +194,7 @@ bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, f
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_block_scores(w.qbar, w.kbar, w.scores, BH, s.N, s.d, p_out, st), "block-score kernel launch");
+  BSA_CUDA(launch_block_scores(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, p_out, st), "block-score kernel launch");
   return BSA_OK;
 }
 
@@ -210,7 +212,7 @@ bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float t
   const int BH = s.B * s.H;
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
+  BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
                          mask_out, w.idx, w.cnt, st),
            "select kernel launch");
   return BSA_OK;
@@ -230,7 +232,7 @@ bsa_status sparse_attn_select_cdf(const void* q, const void* k, bsa_shape s, flo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
            "cdf select kernel launch");
   return BSA_OK;
 }
@@ -253,7 +255,7 @@ bsa_status sparse_attn_cdf(const void* q, const void* k, const void* v, bsa_shap
   const int BH = s.B * s.H;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
            "cdf select kernel launch");
   const char* why = nullptr;
   cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, 0, w.idx, w.cnt, w.status,
@@ -301,7 +303,7 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
+  BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
                          mask_out, w.idx, w.cnt, st),
            "select kernel launch");
   const char* why = nullptr;
@@ -395,7 +397,7 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
       Workspace wc;
       workspace_layout(1, bhc, s.N, s.d, &wc, ws);
       BSA_CUDA(launch_pool(qd + off, kd + off, bhc, s.N, s.d, wc.qbar, wc.kbar, st), "pool kernel launch");
-      BSA_CUDA(launch_select(wc.qbar, wc.kbar, wc.scores, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr,
+      BSA_CUDA(launch_select(wc.qbar, wc.kbar, wc.scores, wc.score_heads, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr,
                              wc.idx, wc.cnt, st),
                "select kernel launch");
       const char* why = nullptr;

@@ -14,13 +14,17 @@ struct Workspace {
   DeviceStatus* status;  // 256 bytes
   float* qbar;           // [B*H, Qb, d]
   float* kbar;           // [B*H, Kb, d]
-  float* scores;         // [B*H, Qb, padded_kb(Kb)]  block dot products Qbar_i . Kbar_j
+  float* scores;         // [score_heads, Qb, padded_kb(Kb)]  block dot products Qbar_i . Kbar_j
+  int score_heads;       // heads whose score matrices the scores section holds at once
   int16_t* idx;          // [B*H, Qb, Kb]  ascending kept key-block indices (prefix of cnt)
   int32_t* cnt;          // [B*H, Qb]
   size_t bytes;
 };
 
-size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base);
+// Carves `base` into the sections above; returns the bytes needed.  The scores
+// section holds score_heads heads at a time (<= 0 or > B*H: all B*H); the
+// selection launchers then work through the heads in chunks of that many.
+size_t workspace_layout(int B, int H, int N, int d, Workspace* ws, void* base, int score_heads = 0);
 
 // Row stride of the block-score matrix: Kb rounded up to a multiple of 4 floats.
 inline int padded_kb(int Kb) { return (Kb + 3) & ~3; }
@@ -38,19 +42,19 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
 // (a3, a4) block scores (into `scores`) and top-k; writes mask (optional), idx
 // and cnt.  kkeep is the kept count per row; with causal != 0 each row i
 // instead keeps ceil(topk * E_i) of its E_i = min(2i+2, Kb) eligible blocks.
-cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int BH, int N, int d,
-                          int kkeep, float topk, int causal, uint8_t* mask_out, int16_t* idx,
-                          int32_t* cnt, cudaStream_t st);
+cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int score_heads, int BH,
+                          int N, int d, int kkeep, float topk, int causal, uint8_t* mask_out,
+                          int16_t* idx, int32_t* cnt, cudaStream_t st);
 
 // cdfthreshd selection: the shortest score-ordered prefix reaching softmax mass
 // `threshold`; writes mask (optional), idx and cnt.
-cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int BH, int N,
-                              int d, float threshold, uint8_t* mask_out, int16_t* idx,
-                              int32_t* cnt, cudaStream_t st);
+cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int score_heads,
+                              int BH, int N, int d, float threshold, uint8_t* mask_out,
+                              int16_t* idx, int32_t* cnt, cudaStream_t st);
 
 // (a3) block-score map only: p_out = softmax of the scaled block scores.
-cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int BH, int N,
-                                int d, float* p_out, cudaStream_t st);
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int score_heads,
+                                int BH, int N, int d, float* p_out, cudaStream_t st);
 
 // (a4') caller mask (NULL = all ones) -> idx and cnt; causal != 0 drops the
 // blocks past 2i+1 of row i.

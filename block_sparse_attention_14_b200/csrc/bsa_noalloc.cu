@@ -65,7 +65,9 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
     if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0)
       return reject(BSA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
   if (!(topk > 0.f) || !(topk <= 1.f)) return reject(BSA_ERR_INVALID_ARG, "topk must lie in (0, 1]");
-  const size_t need = workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr);
+  // The scratch holds the block-score matrices of as many heads at a time as
+  // fit (at least one); the selection then runs over the heads in chunks.
+  const size_t need = workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr, 1);
   if (need > kStaticScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof(msg),
@@ -74,11 +76,16 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
              need, kStaticScratchBytes);
     return reject(BSA_ERR_INVALID_ARG, msg);
   }
+  const int BHs = s.B * s.H;
+  int score_heads = 1;
+  while (score_heads < BHs &&
+         workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr, 2 * score_heads) <= kStaticScratchBytes)
+    score_heads *= 2;
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   Workspace w;
-  workspace_layout(s.B, s.H, s.N, s.d, &w, base);
+  workspace_layout(s.B, s.H, s.N, s.d, &w, base, score_heads);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
@@ -87,7 +94,7 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
   // The status word must start at zero; everything else is overwritten.
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
       (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
-      (e = launch_select(w.qbar, w.kbar, w.scores, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
+      (e = launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
                          w.cnt, st)) != cudaSuccess)
     return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   const char* why = nullptr;

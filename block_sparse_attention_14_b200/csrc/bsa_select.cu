@@ -530,59 +530,82 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int BH, int N, int d,
-                          int kk, float topk, int causal, uint8_t* mask_out, int16_t* idx,
-                          int32_t* cnt, cudaStream_t st) {
+// The selection launchers work through the heads in chunks of score_heads: the
+// dot products of a chunk go to the scores section, then the row kernels of
+// that chunk read them.  Everything is stream-ordered, so chunks reuse it.
+cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int score_heads, int BH,
+                          int N, int d, int kk, float topk, int causal, uint8_t* mask_out,
+                          int16_t* idx, int32_t* cnt, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
-  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
-  if (e != cudaSuccess) return e;
-  const int rows = BH * Qb;
   const size_t smem = row_smem(Kp, true);
-  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  select_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
-      scores, rows, Qb, Kb, Kp, kk, topk, causal, mask_out, idx, cnt);
-  return cudaGetLastError();
+  const int sh = (score_heads <= 0 || score_heads > BH) ? BH : score_heads;
+  for (int h0 = 0; h0 < BH; h0 += sh) {
+    const int nh = BH - h0 < sh ? BH - h0 : sh;
+    const size_t r0 = static_cast<size_t>(h0) * Qb;
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    if (e != cudaSuccess) return e;
+    const int rows = nh * Qb;
+    select_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+        scores, rows, Qb, Kb, Kp, kk, topk, causal, mask_out ? mask_out + r0 * Kb : nullptr,
+        idx + r0 * Kb, cnt + r0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
-cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int BH, int N,
-                              int d, float threshold, uint8_t* mask_out, int16_t* idx,
-                              int32_t* cnt, cudaStream_t st) {
+cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int score_heads,
+                              int BH, int N, int d, float threshold, uint8_t* mask_out,
+                              int16_t* idx, int32_t* cnt, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
-  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
-  if (e != cudaSuccess) return e;
-  const int rows = BH * Qb;
   const size_t smem = row_smem(Kp, false);
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  e = cudaFuncSetAttribute(select_cdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(select_cdf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  select_cdf_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
-      scores, rows, Kb, Kp, scale, threshold, mask_out, idx, cnt);
-  return cudaGetLastError();
+  const int sh = (score_heads <= 0 || score_heads > BH) ? BH : score_heads;
+  for (int h0 = 0; h0 < BH; h0 += sh) {
+    const int nh = BH - h0 < sh ? BH - h0 : sh;
+    const size_t r0 = static_cast<size_t>(h0) * Qb;
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    if (e != cudaSuccess) return e;
+    const int rows = nh * Qb;
+    select_cdf_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+        scores, rows, Kb, Kp, scale, threshold, mask_out ? mask_out + r0 * Kb : nullptr, idx + r0 * Kb,
+        cnt + r0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
-cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int BH, int N,
-                                int d, float* p_out, cudaStream_t st) {
+cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int score_heads,
+                                int BH, int N, int d, float* p_out, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
-  cudaError_t e = launch_dots(qbar, kbar, BH, Qb, Kb, d, scores, st);
-  if (e != cudaSuccess) return e;
-  const int rows = BH * Qb;
   const size_t smem = row_smem(Kp, false);
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  e = cudaFuncSetAttribute(block_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(block_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  block_scores_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
-      scores, rows, Kb, Kp, scale, p_out);
-  return cudaGetLastError();
+  const int sh = (score_heads <= 0 || score_heads > BH) ? BH : score_heads;
+  for (int h0 = 0; h0 < BH; h0 += sh) {
+    const int nh = BH - h0 < sh ? BH - h0 : sh;
+    const size_t r0 = static_cast<size_t>(h0) * Qb;
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    if (e != cudaSuccess) return e;
+    const int rows = nh * Qb;
+    block_scores_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
+        scores, rows, Kb, Kp, scale, p_out + r0 * Kb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_compact(const uint8_t* mask, int BH, int N, int causal, int16_t* idx,

@@ -158,8 +158,10 @@ bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, 
  * start-up (so no memory is left for a workspace), or a caller on a
  * latency-critical path that must not trigger the device-wide synchronisation
  * of cudaFree.  Its scratch is a file-scope device array of 32 MiB, held on
- * every GPU that loads the library until the process exits; shapes whose
- * workspace (bsa_workspace_bytes) exceeds 32 MiB are rejected with
+ * every GPU that loads the library until the process exits.  The scratch holds
+ * the block-score matrices of as many heads at a time as fit (the selection
+ * then runs over the heads in chunks, with the same results); shapes whose
+ * workspace with one head's score matrix exceeds 32 MiB are rejected with
  * BSA_ERR_INVALID_ARG before anything is launched.  The first call on a device
  * looks up that device's copy of the array with cudaGetSymbolAddress (with the
  * device current), so make the first call on each device before any stream

@@ -30,10 +30,16 @@ def _noalloc():
     return f
 
 
-@pytest.mark.parametrize("N,d,topk", [(3001, 128, 0.5), (2500, 64, 0.3)])
-def test_noalloc_matches_fused_call_twice(N, d, topk, cuda_device):
+@pytest.mark.parametrize("B,H,N,d,topk", [
+    (2, 3, 3001, 128, 0.5),
+    (2, 3, 2500, 64, 0.3),
+    # the scratch holds the score matrices of 4 of these 10 heads at a time, so
+    # the selection runs in chunks of 4, 4 and 2 heads
+    (1, 10, 75600, 64, 0.5),
+])
+def test_noalloc_matches_fused_call_twice(B, H, N, d, topk, cuda_device):
     f = _noalloc()
-    wl = W.custom("na", B=2, H=3, d=d, N=N, seed=N + d)
+    wl = W.custom("na", B=B, H=H, d=d, N=N, seed=N + d)
     q, k, v = (t.cuda() for t in W.make_qkv(wl))
     ref_out, ref_mask = bsa.sparse_attn_topk(q, k, v, topk, return_mask=True)
     stream = torch.cuda.current_stream().cuda_stream
