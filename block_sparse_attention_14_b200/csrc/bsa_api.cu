@@ -379,9 +379,19 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
     char* kd = static_cast<char*>(k_dev);
     char* vd = static_cast<char*>(v_dev);
     char* od = static_cast<char*>(out_dev);
+    // With the default chunking the first and the last chunk hold one head each:
+    // the pipeline then fills with one head's copy in and drains with one head's
+    // copy out; the other heads split evenly over the middle chunks.
+    const bool ramp = chunks <= 0 && nc >= 3 && BH >= nc + 2;
+    const auto bound = [&](int c) -> int {
+      if (!ramp) return static_cast<int>(static_cast<int64_t>(BH) * c / nc);
+      if (c == 0) return 0;
+      if (c >= nc) return BH;
+      return 1 + static_cast<int>(static_cast<int64_t>(BH - 2) * (c - 1) / (nc - 2));
+    };
     for (int c = 0; c < nc; ++c) {
-      const int h0 = static_cast<int>(static_cast<int64_t>(BH) * c / nc);
-      const int h1 = static_cast<int>(static_cast<int64_t>(BH) * (c + 1) / nc);
+      const int h0 = bound(c);
+      const int h1 = bound(c + 1);
       const int bhc = h1 - h0;
       if (bhc == 0) continue;
       const size_t off = static_cast<size_t>(h0) * head_bytes;

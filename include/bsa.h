@@ -186,8 +186,10 @@ bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
  *  - q_dev, k_dev, v_dev, out_dev: device buffers of the same size, owned by the
  *    caller; the call overwrites all four.
  *  - ws, ws_bytes: a workspace for the full shape (bsa_workspace_bytes(s)).
- *  - chunks: number of head chunks, clamped to [1, min(B*H, 64)]; <= 0 picks
- *    about eight waves of attention CTAs (one per SM) per chunk.
+ *  - chunks: number of head chunks, clamped to [1, min(B*H, 64)], heads split
+ *    evenly.  <= 0 picks about eight waves of attention CTAs (one per SM) per
+ *    chunk, with one head in the first and in the last chunk (so the pipeline
+ *    fills and drains with one head's copies).
  *  - stream: the compute stream.  Nothing starts before the work already queued
  *    on it, and it waits for the last copy out, so synchronising `stream` (then
  *    bsa_last_device_status) covers the whole call.  Non-causal and causal as in
