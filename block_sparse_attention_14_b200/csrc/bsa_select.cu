@@ -164,10 +164,17 @@ __global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __res
       const float4 kb = *reinterpret_cast<const float4*>(Ks + dd * kDotKs + 128 + 4 * tx);
       const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
       const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      // Two accumulators per packed fma.rn.f32x2: each lane is the same fmaf.
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+      for (int a = 0; a < 8; ++a) {
+        const uint64_t q2 = f2_pack(qv[a], qv[a]);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
+        for (int b = 0; b < 8; b += 2) {
+          uint64_t c2 = f2_pack(acc[a][b], acc[a][b + 1]);
+          c2 = f2_fma(q2, f2_pack(kv[b], kv[b + 1]), c2);
+          f2_unpack(c2, acc[a][b], acc[a][b + 1]);
+        }
+      }
     }
   }
 #pragma unroll
