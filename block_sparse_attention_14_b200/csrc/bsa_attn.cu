@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(384, 1)
       bar_vfull[C::kVSt], bar_vempty[C::kVSt], bar_sfull[2], bar_sfree[2], bar_pfull[2],
       bar_pfree[2], bar_odone, bar_qkdone;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_cnt, s_last, s_fail;
+  __shared__ int s_cnt, s_fail;
   __shared__ int s_tail[4];  // the last four kept key blocks (diagonal blocks are among them)
 
   const int warp = threadIdx.x >> 5;
@@ -131,34 +131,17 @@ __global__ void __launch_bounds__(384, 1)
   const int16_t* idx_row = a.idx + row_id * a.Kb;
   __nv_bfloat16* out_blk = a.out + (static_cast<size_t>(bh) * a.N + static_cast<size_t>(qi) * kBlockQ) * D;
 
-  // One thread reads the count (and whether an earlier CTA already gave up) so
-  // that every thread takes the same early-exit decision.
-  if (threadIdx.x == 0) {
-    const int c = (*reinterpret_cast<volatile uint32_t*>(&a.status->code) != 0) ? -1 : a.cnt[row_id];
-    s_cnt = c;
-    s_last = c > 0 ? idx_row[c - 1] : -1;  // the ragged last key block can only be the last kept one
-    s_fail = 0;
-    if (kCausal) {
-#pragma unroll
-      for (int t = 0; t < 4; ++t) s_tail[t] = (c - 4 + t >= 0) ? idx_row[c - 4 + t] : -1;
-    }
-  }
-  __syncthreads();
-  const int cnt = s_cnt;
-  if (cnt < 0) return;
-  if (cnt == 0) {  // no kept key block: the defined output is zero
-    uint4* o4 = reinterpret_cast<uint4*>(out_blk);
-    for (int e = threadIdx.x; e < rows_valid * D / 8; e += blockDim.x) o4[e] = make_uint4(0, 0, 0, 0);
-    return;
-  }
-
   const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
   const uint32_t sQ = base;
   const uint32_t sK0 = base + C::kOffK;
   const uint32_t sV0 = base + C::kOffV;
   const uint32_t sP0 = base + C::kOffP;
 
+  // Thread 0 initialises the barriers and reads the count (and whether an
+  // earlier CTA already gave up) while warp 1 allocates TMEM; every thread then
+  // takes the same early-exit decision.
   if (threadIdx.x == 0) {
+    const int c = (*reinterpret_cast<volatile uint32_t*>(&a.status->code) != 0) ? -1 : a.cnt[row_id];
     mbar_init(smem_u32(&bar_q), 1);
     for (int s = 0; s < C::kKSt; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
@@ -177,6 +160,12 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(&bar_odone), 1);
     mbar_init(smem_u32(&bar_qkdone), 1);
     fence_mbar_init();
+    s_cnt = c;
+    s_fail = 0;
+    if (kCausal) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) s_tail[t] = (c - 4 + t >= 0) ? idx_row[c - 4 + t] : -1;
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);
@@ -185,6 +174,15 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int cnt = s_cnt;
+  if (cnt <= 0) {
+    if (cnt == 0) {  // no kept key block: the defined output is zero
+      uint4* o4 = reinterpret_cast<uint4*>(out_blk);
+      for (int e = threadIdx.x; e < rows_valid * D / 8; e += blockDim.x) o4[e] = make_uint4(0, 0, 0, 0);
+    }
+    if (warp == 1) tmem_dealloc(s_tmem, C::kTmemCols);
+    return;
+  }
   const uint32_t tmem = s_tmem;
   const int npairs = (cnt + 1) >> 1;
   DeviceStatus* st = a.status;
@@ -212,6 +210,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_3d(sQ + c * C::kChunk, &tm_q, smem_u32(&bar_q), c * 64, qi * kBlockQ, bh);
+        // The CTA that this SM is likely to run next (one per SM, dispatched in
+        // order) starts with a Q tile from HBM; bring it into L2 now.
+        uint32_t nsm;
+        asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+        const unsigned nxt = blockIdx.x + nsm;
+        if (nxt < gridDim.x) {
+          const int nbh = static_cast<int>(nxt / a.Qb), nqi = static_cast<int>(nxt - nbh * a.Qb);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) tma_prefetch_l2_3d(&tm_q, c * 64, nqi * kBlockQ, nbh);
+        }
       }
       int b0 = __ldg(idx_row), b1 = cnt > 1 ? __ldg(idx_row + 1) : 0;
       for (int j = 0; j < npairs; ++j) {
@@ -316,7 +324,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     const int kb_last = a.Kb - 1;
     const int tail = a.N - kb_last * kBlockK;  // valid keys in the last key block (1..64)
-    const bool ragged = tail < 64 && s_last == kb_last;
+    // The ragged last key block can only be the last kept one.
+    const bool ragged = tail < 64 && __ldg(idx_row + cnt - 1) == kb_last;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int t = 0;

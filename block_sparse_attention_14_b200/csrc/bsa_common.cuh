@@ -115,6 +115,15 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Prefetches one box of a 3-D tensor map into L2 (no shared-memory destination,
+// no completion to wait for).  Same coordinate rules as tma_load_3d.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // 3-D tiled bulk load global -> shared, completion counted on `bar` in bytes.
 // x is the innermost (element) coordinate; callers keep x * 2 bytes a multiple
 // of 16 (x is 0 or 64 here).
