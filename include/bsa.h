@@ -23,11 +23,14 @@
  *  - Qb = ceil(N / 128), Kb = ceil(N / 64).  N <= 131072, so Kb <= 2048.
  *  - mask tensors are uint8 [B, H, Qb, Kb], row-major; nonzero means "keep".
  *  - ws: a device workspace of at least bsa_workspace_bytes(shape) bytes,
- *    256-byte aligned, owned by the caller.  The library never allocates and
- *    keeps no per-call state between calls; calls that share one workspace must
- *    be ordered on one stream.
+ *    256-byte aligned, owned by the caller.  The library never allocates device
+ *    memory and keeps no per-call state between calls (sparse_attn_topk_host
+ *    creates, and releases, two copy streams and their events per call); calls
+ *    that share one workspace must be ordered on one stream.
  *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
- *    Every call is asynchronous on it and returns after launching.
+ *    Every call is asynchronous on it and returns after launching (for
+ *    sparse_attn_topk_host the host buffers must stay valid until `stream` has
+ *    been synchronised).
  *  - The attention scale is 1/sqrt(d), as in scaled-dot-product attention.
  *  - Errors: arguments are validated on the host before anything is launched;
  *    a rejected call returns BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED and
