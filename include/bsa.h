@@ -7,8 +7,9 @@
  *   (1) selection: mean-pool q over 128-row blocks and k over 64-row blocks,
  *       score the blocks with softmax(Qbar Kbar^T / sqrt(d)) per head, and keep
  *       the top-k fraction of key blocks for every query block;
- *   (2) attention: non-causal softmax attention that visits only the kept
- *       128 x 64 tiles.
+ *   (2) attention: softmax attention that visits only the kept 128 x 64
+ *       tiles (non-causal by default; is_causal != 0 restricts each row to
+ *       keys at or before its own position).
  *
  * The calls mirror the interface on "SpargeAttention Documentation":
  * spas_sage2_attn_meansim_topk_cuda(q, k, v, topk, is_causal) (recommended API
