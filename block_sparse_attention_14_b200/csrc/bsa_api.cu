@@ -52,6 +52,22 @@ bsa_status check_tensor(const void* p, const char* name) {
   return BSA_OK;
 }
 
+// out must not overlap q, k or v: every CTA of a head reads that head's K and
+// V while other CTAs write their output rows.
+bsa_status check_out_disjoint(const bsa_shape& s, const void* out, const void* q, const void* k,
+                              const void* v) {
+  const size_t bytes = static_cast<size_t>(s.B) * s.H * s.N * s.d * 2;
+  const uintptr_t o = reinterpret_cast<uintptr_t>(out);
+  const void* ins[3] = {q, k, v};
+  const char* names[3] = {"q", "k", "v"};
+  for (int i = 0; i < 3; ++i) {
+    const uintptr_t p = reinterpret_cast<uintptr_t>(ins[i]);
+    if (o < p + bytes && p < o + bytes)
+      return fail(BSA_ERR_INVALID_ARG, "out overlaps %s; the attention output needs its own buffer", names[i]);
+  }
+  return BSA_OK;
+}
+
 bsa_status check_ws(const bsa_shape& s, void* ws, size_t ws_bytes, Workspace* out) {
   if (ws == nullptr) return fail(BSA_ERR_INVALID_ARG, "workspace is NULL");
   if (!aligned(ws, 256)) return fail(BSA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
@@ -247,6 +263,7 @@ bsa_status sparse_attn_cdf(const void* q, const void* k, const void* v, bsa_shap
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
   BSA_TRY(check_tensor(out, "out"));
+  BSA_TRY(check_out_disjoint(s, out, q, k, v));
   if (!(threshold > 0.f) || !(threshold <= 1.f))
     return fail(BSA_ERR_INVALID_ARG, "threshold must lie in (0, 1] (got %g)", static_cast<double>(threshold));
   Workspace w;
@@ -273,6 +290,7 @@ bsa_status block_sparse_attn_fwd(const void* q, const void* k, const void* v, bs
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
   BSA_TRY(check_tensor(out, "out"));
+  BSA_TRY(check_out_disjoint(s, out, q, k, v));
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -295,6 +313,7 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
   BSA_TRY(check_tensor(out, "out"));
+  BSA_TRY(check_out_disjoint(s, out, q, k, v));
   BSA_TRY(check_topk(topk));
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
@@ -327,6 +346,7 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
   BSA_TRY(check_tensor(k_dev, "k_dev"));
   BSA_TRY(check_tensor(v_dev, "v_dev"));
   BSA_TRY(check_tensor(out_dev, "out_dev"));
+  BSA_TRY(check_out_disjoint(s, out_dev, q_dev, k_dev, v_dev));
   BSA_TRY(check_topk(topk));
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
@@ -448,6 +468,7 @@ bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, 
   BSA_TRY(check_tensor(k, "k"));
   BSA_TRY(check_tensor(v, "v"));
   BSA_TRY(check_tensor(out, "out"));
+  BSA_TRY(check_out_disjoint(s, out, q, k, v));
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);

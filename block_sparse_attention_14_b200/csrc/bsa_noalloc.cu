@@ -65,6 +65,15 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
     if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0)
       return reject(BSA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
   if (!(topk > 0.f) || !(topk <= 1.f)) return reject(BSA_ERR_INVALID_ARG, "topk must lie in (0, 1]");
+  {
+    const size_t bytes = static_cast<size_t>(s.B) * s.H * s.N * s.d * 2;
+    const uintptr_t o = reinterpret_cast<uintptr_t>(out);
+    for (const void* in : {q, k, v}) {
+      const uintptr_t p = reinterpret_cast<uintptr_t>(in);
+      if (o < p + bytes && p < o + bytes)
+        return reject(BSA_ERR_INVALID_ARG, "out overlaps q, k or v; the attention output needs its own buffer");
+    }
+  }
   // The scratch holds the block-score matrices of as many heads at a time as
   // fit (at least one); the selection then runs over the heads in chunks.
   const size_t need = workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr, 1);

@@ -21,6 +21,7 @@
  * Conventions shared by every call
  *  - q, k, v, out: device pointers to contiguous bf16 tensors of shape
  *    [B, H, N, d] (row-major, d fastest), 16-byte aligned.  d is 64 or 128.
+ *    out must not overlap q, k or v (BSA_ERR_INVALID_ARG).
  *  - Qb = ceil(N / 128), Kb = ceil(N / 64).  N <= 131072, so Kb <= 2048.
  *  - mask tensors are uint8 [B, H, Qb, Kb], row-major; nonzero means "keep".
  *  - ws: a device workspace of at least bsa_workspace_bytes(shape) bytes,

@@ -48,12 +48,33 @@ def test_workspace_bytes():
         assert bsa.workspace_bytes(*bad) == 0
 
 
-def _call_topk(shape, topk=0.5, is_causal=0, q=256, k=256, v=256, out=256, ws=512, ws_bytes=None):
+# Distinct fake device addresses, far enough apart that no tensor of the shapes
+# used here overlaps another (nothing is launched: every call is rejected on the host).
+QA, KA, VA, OA = 1 << 30, (1 << 30) + (1 << 26), (1 << 30) + (2 << 26), (1 << 30) + (3 << 26)
+
+
+def _call_topk(shape, topk=0.5, is_causal=0, q=QA, k=KA, v=VA, out=OA, ws=512, ws_bytes=None):
     L = bsa.lib()
     s = bsa.Shape(*shape)
     if ws_bytes is None:
         ws_bytes = L.bsa_workspace_bytes(s)
     return L.sparse_attn_topk(q, k, v, s, topk, is_causal, out, None, ws, ws_bytes, None)
+
+
+def test_output_must_not_overlap_inputs():
+    L = bsa.lib()
+    s = bsa.Shape(1, 1, 128, 64)          # 16 KiB per tensor
+    n = L.bsa_workspace_bytes(s)
+    base = 1 << 20
+    q, k, v, ws = base, base + (1 << 16), base + (2 << 16), base + (4 << 16)
+    for out in (q, k + 4096, v - 4096):   # same as q, inside k, straddling into v
+        assert L.sparse_attn_topk(q, k, v, s, 0.5, 0, out, None, ws, n, None) == 1
+        assert b"overlaps" in L.bsa_last_error_message()
+        assert L.block_sparse_attn_fwd(q, k, v, s, None, 0, out, ws, n, None) == 1
+        assert L.block_sparse_attn_apply(q, k, v, s, 0, out, ws, n, None) == 1
+    L.sparse_attn_topk_noalloc.argtypes = [ctypes.c_void_p] * 3 + [bsa.Shape, ctypes.c_float, ctypes.c_int] + [ctypes.c_void_p] * 3
+    L.sparse_attn_topk_noalloc.restype = ctypes.c_int
+    assert L.sparse_attn_topk_noalloc(q, k, v, s, 0.5, 0, k, None, None) == 1
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -64,14 +85,15 @@ def _call_topk(shape, topk=0.5, is_causal=0, q=256, k=256, v=256, out=256, ws=51
     (dict(shape=(1, 1, 128, 64), topk=1.5), 1),
     (dict(shape=(1, 1, 128, 64), topk=float("nan")), 1),
     (dict(shape=(1, 1, 128, 64), q=None), 1),
-    (dict(shape=(1, 1, 128, 64), v=264), 1),        # unaligned pointer
+    (dict(shape=(1, 1, 128, 64), v=VA + 8), 1),     # unaligned pointer
     (dict(shape=(1, 1, 128, 64), ws=None), 1),
     (dict(shape=(1, 1, 128, 64), ws=512 + 16), 1),  # workspace not 256-aligned
     (dict(shape=(1, 1, 128, 64), ws_bytes=100), 1),  # workspace too small
 ])
 def test_fused_call_rejects_bad_arguments(kw, code):
     assert _call_topk(**kw) == code
-    assert bsa.lib().bsa_last_error_message().decode() != ""
+    msg = bsa.lib().bsa_last_error_message().decode()
+    assert msg != "" and "overlaps" not in msg
 
 
 def test_other_calls_reject_bad_arguments():
@@ -115,6 +137,7 @@ def test_cdf_calls_reject_bad_thresholds():
     n = L.bsa_workspace_bytes(s)
     for bad in (0.0, -0.5, 1.5, float("nan")):
         assert L.sparse_attn_select_cdf(256, 256, s, bad, 1024, 512, n, None) == 1
-        assert L.sparse_attn_cdf(256, 256, 256, s, bad, 0, 256, None, 512, n, None) == 1
-    assert L.sparse_attn_cdf(256, 256, 256, s, 0.9, 1, 256, None, 512, n, None) == 2
+        assert L.sparse_attn_cdf(QA, KA, VA, s, bad, 0, OA, None, 512, n, None) == 1
+        assert b"threshold" in L.bsa_last_error_message()
+    assert L.sparse_attn_cdf(QA, KA, VA, s, 0.9, 1, OA, None, 512, n, None) == 2
     assert L.sparse_attn_select_cdf(256, 256, s, 0.9, None, 512, n, None) == 1

@@ -58,8 +58,9 @@ def test_noalloc_matches_fused_call_twice(B, H, N, d, topk, cuda_device):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):
     f = _noalloc()
-    q = torch.zeros(16, dtype=torch.bfloat16, device="cuda")  # never read: rejected before launch
-    p = q.data_ptr()
-    st = f(p, p, p, bsa.Shape(1, 40, 75600, 128), 0.5, 0, p, None, None)
+    # Distinct, never-dereferenced addresses 1 GiB apart (each tensor of this shape
+    # is 774 MB): the call is rejected on the host before anything is launched.
+    q, k, v, out = (g << 30 for g in (4, 5, 6, 7))
+    st = f(q, k, v, bsa.Shape(1, 40, 75600, 128), 0.5, 0, out, None, None)
     assert st == 1
     assert "static scratch" in bsa.lib().bsa_last_error_message().decode()
