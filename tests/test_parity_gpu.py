@@ -237,3 +237,26 @@ def test_cdf_selection_and_attention_match_oracle(N, d, tau, cuda_device):
     same = np.all(m1.cpu().numpy() == mref, axis=-1)
     rows = np.repeat(same, 128, axis=2)[:, :, :N]
     assert_close(out.float().cpu().numpy()[rows], ref[rows], f"cdf {N,d,tau}")
+
+
+@pytest.mark.parametrize("N,d,scale,causal,order", [(3000, 128, 4.0, False, "ascending"),
+                                                    (3000, 64, 4.0, False, "ascending"),
+                                                    (2500, 128, 4.0, True, "ascending"),
+                                                    (3000, 128, 3.0, False, "random")])
+def test_large_score_jumps_rescale_exactly(N, d, scale, causal, order, cuda_device):
+    """Scores of tens to ~100 in log2 units that grow from one kept pair to the next:
+    the running reference maximum is raised, and O and l rescaled, many times per
+    row; the result must still match the fp64 oracle.  (Much larger scores make the
+    fp32 accumulation of the tensor-core Q K^T product, not the softmax, the limit:
+    at q, k ~ N(0, 36) with d = 64 the max-abs error reaches ~3e-2.)"""
+    q, k, v = _qkv(1, 2, N, d, seed=N + d, scale=scale)
+    if order == "ascending":
+        # make later key blocks score higher for every query: add a ramp along the keys
+        ramp = torch.linspace(0.0, 3.0 * scale, N).view(1, 1, N, 1)
+        k = (k.float() + ramp * q.float().mean(dim=2, keepdim=True).sign()).to(torch.bfloat16)
+    out = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), None, is_causal=causal)
+    torch.cuda.synchronize()
+    Qb, Kb = O.block_counts(N)
+    ones = np.ones((1, 2, Qb, Kb), dtype=np.uint8)
+    ref = O.block_sparse_attention(q, k, v, ones, causal=causal)
+    assert_close(out.float().cpu().numpy(), ref, f"large score jumps {N, d, scale, causal, order}")
