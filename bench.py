@@ -47,7 +47,8 @@ from block_sparse_attention_14_b200 import workloads as W  # noqa: E402
 METRIC = "ms/call and dense-equiv TFLOPS, Wan-14B-shaped topk=0.5, % of bf16 TC peak"
 UNIT = "dense-equiv TFLOPS"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_14_b200", "csrc", "bsa_attn.cu")
+ATTN_SRCS = [os.path.join(ROOT, "block_sparse_attention_14_b200", "csrc", f)
+             for f in ("bsa_attn.cu", "bsa_common.cuh")]
 TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "bsa_fwd_kernel_*_ncu.md")
 
 
@@ -77,8 +78,13 @@ def load_peaks():
 
 
 def attn_source_hash() -> str:
-    with open(ATTN_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256[:16] of the attention kernel's sources (the kernel file and the
+    device-helper header it inlines), concatenated."""
+    h = hashlib.sha256()
+    for path in ATTN_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
