@@ -120,8 +120,8 @@ bsa_status check_pinned(const void* p, const char* name) {
 // Streams and events of one host-pipelined call.  Destroying them while work
 // is still pending is allowed: CUDA releases them once that work completes.
 struct PipelineResources {
-  cudaStream_t copy_in = nullptr, copy_out = nullptr;
-  cudaEvent_t events[2 + 2 * 64] = {};
+  cudaStream_t copy_in = nullptr, copy_out = nullptr, select = nullptr, attn[2] = {nullptr, nullptr};
+  cudaEvent_t events[2 + 3 * 64] = {};
   int n_events = 0;
   cudaError_t event(cudaEvent_t* e) {
     cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
@@ -132,6 +132,9 @@ struct PipelineResources {
     for (int i = 0; i < n_events; ++i) cudaEventDestroy(events[i]);
     if (copy_in) cudaStreamDestroy(copy_in);
     if (copy_out) cudaStreamDestroy(copy_out);
+    if (select) cudaStreamDestroy(select);
+    for (cudaStream_t a : attn)
+      if (a) cudaStreamDestroy(a);
   }
 };
 
@@ -359,15 +362,16 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
   const int max_chunks = BH < 64 ? BH : 64;
   int nc = chunks;
   if (nc <= 0) {
-    // About eight waves of attention CTAs (one per SM) per chunk: enough to keep
-    // the tail of each chunk small, small enough to keep the pipeline's fill
-    // and drain (one chunk's copy in and copy out) short.
+    // About four waves of attention CTAs (one per SM) per chunk.  A chunk's last
+    // wave overlaps the next chunk's selection and first CTAs, so small chunks
+    // cost little on the GPU and keep the pipeline's fill and drain (one
+    // chunk's copy in and copy out) short.
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       sms = 148;
     const int64_t ctas = static_cast<int64_t>(BH) * Qb;
-    nc = static_cast<int>((ctas + 4 * sms) / (8 * sms));
+    nc = static_cast<int>((ctas + 2 * sms) / (4 * sms));
   }
   nc = nc < 1 ? 1 : (nc > max_chunks ? max_chunks : nc);
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
@@ -377,19 +381,27 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
 
   PipelineResources r;
   cudaEvent_t e_start = nullptr, e_end = nullptr;
+  int prio_low = 0, prio_high = 0;
+  BSA_CUDA(cudaDeviceGetStreamPriorityRange(&prio_low, &prio_high), "stream priorities");
   BSA_CUDA(cudaStreamCreateWithFlags(&r.copy_in, cudaStreamNonBlocking), "copy stream");
   BSA_CUDA(cudaStreamCreateWithFlags(&r.copy_out, cudaStreamNonBlocking), "copy stream");
+  BSA_CUDA(cudaStreamCreateWithPriority(&r.select, cudaStreamNonBlocking, prio_high), "select stream");
+  for (cudaStream_t& a : r.attn) BSA_CUDA(cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking), "attention stream");
   BSA_CUDA(r.event(&e_start), "event");
   BSA_CUDA(r.event(&e_end), "event");
-  // Nothing of this call starts before the work already queued on `stream`.
-  BSA_CUDA(cudaEventRecord(e_start, st), "event record");
-  BSA_CUDA(cudaStreamWaitEvent(r.copy_in, e_start, 0), "stream wait");
-  BSA_CUDA(cudaStreamWaitEvent(r.copy_out, e_start, 0), "stream wait");
+  // Nothing of this call starts before the work already queued on `stream`
+  // (the status reset included).
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
+  BSA_CUDA(cudaEventRecord(e_start, st), "event record");
+  for (cudaStream_t x : {r.copy_in, r.copy_out, r.select, r.attn[0], r.attn[1]})
+    BSA_CUDA(cudaStreamWaitEvent(x, e_start, 0), "stream wait");
 
-  // Chunk c: heads [h0, h1) of the flattened B*H; copy in on copy_in, compute on
-  // `stream` with the chunk's own workspace layout (status word at offset 0 in
-  // every layout), copy out on copy_out.  Chunks are disjoint byte ranges.
+  // Chunk c: heads [h0, h1) of the flattened B*H.  Copy in on copy_in; selection
+  // on the high-priority select stream, into the chunk's own heads of the full
+  // workspace layout; attention on attn[c % 2]; copy out on copy_out.  Chunks
+  // touch disjoint byte ranges of every buffer, so the selection of chunk c+1
+  // runs on the SMs that chunk c's attention leaves idle in its last wave, and
+  // chunk c+1's attention starts on SMs as chunk c's last CTAs retire.
   const auto run = [&]() -> bsa_status {
     const char* qh = static_cast<const char*>(q_host);
     const char* kh = static_cast<const char*>(k_host);
@@ -416,25 +428,33 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
       if (bhc == 0) continue;
       const size_t off = static_cast<size_t>(h0) * head_bytes;
       const size_t bytes = static_cast<size_t>(bhc) * head_bytes;
-      cudaEvent_t e_in = nullptr, e_done = nullptr;
+      cudaEvent_t e_in = nullptr, e_sel = nullptr, e_done = nullptr;
       BSA_CUDA(r.event(&e_in), "event");
+      BSA_CUDA(r.event(&e_sel), "event");
       BSA_CUDA(r.event(&e_done), "event");
       BSA_CUDA(cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "q copy in");
       BSA_CUDA(cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "k copy in");
       BSA_CUDA(cudaMemcpyAsync(vd + off, vh + off, bytes, cudaMemcpyHostToDevice, r.copy_in), "v copy in");
       BSA_CUDA(cudaEventRecord(e_in, r.copy_in), "event record");
-      BSA_CUDA(cudaStreamWaitEvent(st, e_in, 0), "stream wait");
-      Workspace wc;
-      workspace_layout(1, bhc, s.N, s.d, &wc, ws);
-      BSA_CUDA(launch_pool(qd + off, kd + off, bhc, s.N, s.d, wc.qbar, wc.kbar, st), "pool kernel launch");
-      BSA_CUDA(launch_select(wc.qbar, wc.kbar, wc.scores, wc.score_heads, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr,
-                             wc.idx, wc.cnt, st),
+      BSA_CUDA(cudaStreamWaitEvent(r.select, e_in, 0), "stream wait");
+      const size_t hh = static_cast<size_t>(h0);
+      float* qbar = w.qbar + hh * Qb * s.d;
+      float* kbar = w.kbar + hh * Kb * s.d;
+      float* scores = w.scores + hh * Qb * padded_kb(Kb);
+      int16_t* idx = w.idx + hh * Qb * Kb;
+      int32_t* cnt = w.cnt + hh * Qb;
+      BSA_CUDA(launch_pool(qd + off, kd + off, bhc, s.N, s.d, qbar, kbar, r.select), "pool kernel launch");
+      BSA_CUDA(launch_select(qbar, kbar, scores, bhc, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr, idx, cnt,
+                             r.select),
                "select kernel launch");
+      BSA_CUDA(cudaEventRecord(e_sel, r.select), "event record");
+      cudaStream_t sa = r.attn[c & 1];
+      BSA_CUDA(cudaStreamWaitEvent(sa, e_sel, 0), "stream wait");
       const char* why = nullptr;
       cudaError_t e = launch_attention(qd + off, kd + off, vd + off, od + off, bhc, s.N, s.d, is_causal != 0,
-                                       wc.idx, wc.cnt, wc.status, g_timeout_ns.load(), st, &why);
+                                       idx, cnt, w.status, g_timeout_ns.load(), sa, &why);
       if (e != cudaSuccess) return why ? fail(BSA_ERR_CUDA, "%s", why) : cuda_fail(e, "attention kernel launch");
-      BSA_CUDA(cudaEventRecord(e_done, st), "event record");
+      BSA_CUDA(cudaEventRecord(e_done, sa), "event record");
       BSA_CUDA(cudaStreamWaitEvent(r.copy_out, e_done, 0), "stream wait");
       BSA_CUDA(cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, r.copy_out), "out copy");
     }

@@ -179,8 +179,12 @@ bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
                                     void* stream);
 
 /* sparse_attn_topk on HOST buffers, pipelined over chunks of heads: while the
- * kernels of chunk c run on `stream`, chunk c+1's q/k/v are copied in on one
- * internal copy stream and chunk c-1's output is copied out on another.  The
+ * attention of chunk c runs, chunk c+1's q/k/v are copied in on one internal
+ * copy stream and chunk c-1's output is copied out on another.  Each chunk's
+ * selection runs on a high-priority internal stream as soon as its inputs have
+ * arrived, and the attention of consecutive chunks alternates between two
+ * internal streams, so the next chunk's selection and first attention CTAs take
+ * the SMs that the current chunk's last wave leaves idle.  The
  * pages have no counterpart: heads are independent (the same selection and
  * attention run per head), so this only overlaps PCIe transfers with the
  * compute of sparse_attn_topk, and out_host receives exactly the bytes that
@@ -191,14 +195,17 @@ bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v,
  *  - q_dev, k_dev, v_dev, out_dev: device buffers of the same size, owned by the
  *    caller; the call overwrites all four.
  *  - ws, ws_bytes: a workspace for the full shape (bsa_workspace_bytes(s)).
+ *    Each chunk's selection writes that chunk's heads of it, so afterwards it
+ *    holds the kept-block lists of every head, as after sparse_attn_topk.
  *  - chunks: number of head chunks, clamped to [1, min(B*H, 64)], heads split
- *    evenly.  <= 0 picks about eight waves of attention CTAs (one per SM) per
- *    chunk, with one head in the first and in the last chunk (so the pipeline
- *    fills and drains with one head's copies).
+ *    evenly.  <= 0 picks about four waves of attention CTAs (one per SM) per
+ *    chunk, with one head in the first and in the last chunk when there are at
+ *    least two heads more than chunks (so the pipeline fills and drains with one
+ *    head's copies).
  *  - stream: the compute stream.  Nothing starts before the work already queued
  *    on it, and it waits for the last copy out, so synchronising `stream` (then
  *    bsa_last_device_status) covers the whole call.  Non-causal and causal as in
- *    sparse_attn_topk; no mask is written.  The call creates two streams and
+ *    sparse_attn_topk; no mask is written.  The call creates five streams and
  *    their events and releases them when the work completes, so calls from
  *    several host threads do not share state. */
 bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const void* v_host,

@@ -52,3 +52,31 @@ def test_host_pipeline_rejects_pageable_memory(cuda_device):
                                  *[t.data_ptr() for t in dev], ws.data_ptr(), ws.numel(), 0, None)
     assert st == 1
     assert b"page-locked" in L.bsa_last_error_message()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal,chunks", [(False, 0), (True, 3)])
+def test_host_pipeline_leaves_every_heads_lists_in_the_workspace(cuda_device, causal, chunks):
+    """Each chunk's selection writes its own heads of the full workspace layout, so
+    after the call the kept-block lists of all heads are there, equal to those
+    sparse_attn_topk leaves."""
+    import numpy as np
+
+    from tests.parity import workspace_lists
+
+    B, H, N, d = 1, 7, 2900, 128
+    q, k, v = _case(B, H, N, d, seed=77)
+    ws_dev, ws_host = bsa.make_workspace(B, H, N, d), bsa.make_workspace(B, H, N, d)
+    ref = bsa.sparse_attn_topk(q.cuda(), k.cuda(), v.cuda(), 0.3, causal, workspace=ws_dev)
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    bufs = tuple(torch.empty_like(ref) for _ in range(4))
+    out = bsa.sparse_attn_topk_host(qp, kp, vp, 0.3, causal, device_buffers=bufs, workspace=ws_host,
+                                    chunks=chunks)
+    bsa.last_device_status(ws_host)
+    assert torch.equal(out, ref.cpu())
+    Qb, Kb = (N + 127) // 128, (N + 63) // 64
+    idx_d, cnt_d = workspace_lists(ws_dev, B * H, Qb, Kb, d)
+    idx_h, cnt_h = workspace_lists(ws_host, B * H, Qb, Kb, d)
+    assert np.array_equal(cnt_h, cnt_d)
+    valid = np.arange(Kb)[None, :] < cnt_d[:, None]
+    assert np.array_equal(np.where(valid, idx_h, -1), np.where(valid, idx_d, -1))
