@@ -27,7 +27,7 @@
  *  - ws: a device workspace of at least bsa_workspace_bytes(shape) bytes,
  *    256-byte aligned, owned by the caller.  The library never allocates device
  *    memory and keeps no per-call state between calls (sparse_attn_topk_host
- *    creates, and releases, two copy streams and their events per call); calls
+ *    creates, and releases, five streams and their events per call); calls
  *    that share one workspace must be ordered on one stream.
  *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous on it and returns after launching (for
