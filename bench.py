@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+from datetime import datetime
 import glob
 import hashlib
 import io
@@ -103,9 +104,11 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples nvidia-smi clocks and throttle reasons every 50 ms.  Started before
+    the warm-up (nvidia-smi takes a few hundred ms to emit its first row); stop()
+    keeps the rows whose timestamps fall inside the timed region."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -123,14 +126,14 @@ class ClockSampler:
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
             if self.bus:
                 cmd.insert(1, f"--id={self.bus}")
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin: float, t_end: float):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -141,9 +144,18 @@ class ClockSampler:
         rows = []
         with open(self.path) as f:
             for r in csv.reader(f):
-                if len(r) >= 8:
-                    rows.append([x.strip() for x in r])
+                if len(r) >= 9:
+                    try:
+                        ts = datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    except ValueError:
+                        continue
+                    rows.append((ts, [x.strip() for x in r[1:]]))
         os.unlink(self.path)
+        timed = [r for ts, r in rows if t_begin <= ts <= t_end]
+        window = "timed region"
+        if not timed:  # the timed region ended before nvidia-smi's first row
+            timed, window = [r for _, r in rows], "whole run"
+        rows = timed
         if not rows:
             return None
         sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
@@ -152,7 +164,8 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
         loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "window": window}
 
 
 def dist_setup():
@@ -286,16 +299,17 @@ def run_b200(args, world, rank, local):
         bsa.sparse_attn_select(q, k, args.topk, mask_out=mask, workspace=ws)
         bsa.block_sparse_attn_apply(q, k, v, ws, out=out)
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(Wm):
         step()
     bsa.last_device_status(ws)
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
-    clocks.start()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
+    t_begin = time.time()
     for i in range(K):
         ev[i][0].record(stream)
         bsa.sparse_attn_select(q, k, args.topk, mask_out=mask, workspace=ws)
@@ -303,8 +317,9 @@ def run_b200(args, world, rank, local):
         bsa.block_sparse_attn_apply(q, k, v, ws, out=out)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
+    t_end = time.time()
     barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop(t_begin, t_end)
     bsa.last_device_status(ws)
     step_s = ev[0][0].elapsed_time(ev[K - 1][2]) / 1e3 / K
     sel_s = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
