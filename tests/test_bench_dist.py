@@ -1,5 +1,6 @@
-"""The benchmark's multi-rank logic on CPU: two gloo ranks, max-over-ranks timing,
-weak-scaling throughput, and the reference arm's rank-0-only rule."""
+"""The benchmark's host logic on CPU: two gloo ranks, max-over-ranks timing,
+weak-scaling throughput, the reference arm's rank-0-only rule, and the clock record's
+restriction to the timed region."""
 import os
 import socket
 
@@ -64,3 +65,52 @@ def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
 def test_single_rank_helpers():
     assert bench.max_over_ranks(0.123, 1) == 0.123
     assert bench.whole_job_value(2e12, 0.5, 1) == pytest.approx(4.0)
+
+
+def _fake_smi(path, rows):
+    with open(path, "w") as f:
+        for ts, mhz, reasons in rows:
+            stamp = ts.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            flags = ", ".join("Active" if r else "Not Active" for r in reasons)
+            f.write(f"{stamp}, {mhz}, 1965, 900.00, 0x4, {flags}\n")
+
+
+class _DoneProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        pass
+
+
+def test_clock_sampler_keeps_only_the_timed_region(tmp_path):
+    """Rows before and after the timed region (warm-up, teardown) are dropped; the
+    median and the throttle reasons come from the rows inside it."""
+    from datetime import datetime, timedelta
+
+    t0 = datetime(2026, 1, 1, 12, 0, 0)
+    cap = (False, False, False, True)
+    thermal = (False, True, False, True)
+    _fake_smi(tmp_path / "smi.csv", [
+        (t0 - timedelta(seconds=1), 1965, thermal),   # warm-up, throttled: dropped
+        (t0 + timedelta(milliseconds=100), 1500, cap),
+        (t0 + timedelta(milliseconds=150), 1480, cap),
+        (t0 + timedelta(milliseconds=200), 1520, cap),
+        (t0 + timedelta(seconds=3), 900, thermal),    # after the region: dropped
+    ])
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.proc, c.path = _DoneProc(), str(tmp_path / "smi.csv")
+    rec = c.stop(t0.timestamp(), (t0 + timedelta(milliseconds=500)).timestamp())
+    assert rec == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3, "window": "timed region"}
+
+
+def test_clock_sampler_falls_back_to_the_whole_run(tmp_path):
+    from datetime import datetime, timedelta
+
+    t0 = datetime(2026, 1, 1, 12, 0, 0)
+    _fake_smi(tmp_path / "smi.csv", [(t0 + timedelta(seconds=2), 1400, (False, False, False, True))])
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.proc, c.path = _DoneProc(), str(tmp_path / "smi.csv")
+    rec = c.stop(t0.timestamp(), (t0 + timedelta(seconds=1)).timestamp())
+    assert rec["window"] == "whole run" and rec["samples"] == 1 and rec["sm_mhz"] == 1400.0
