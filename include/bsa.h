@@ -32,7 +32,11 @@
  *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous on it and returns after launching (for
  *    sparse_attn_topk_host the host buffers must stay valid until `stream` has
- *    been synchronised).
+ *    been synchronised).  The device-buffer calls only enqueue work on `stream`
+ *    and neither allocate nor synchronise, so they may be captured into a CUDA
+ *    graph and replayed (sparse_attn_topk_host synchronises nothing either, but
+ *    creates streams, so it is not meant for capture; bsa_last_device_status
+ *    synchronises `stream`).
  *  - The attention scale is 1/sqrt(d), as in scaled-dot-product attention.
  *  - Errors: arguments are validated on the host before anything is launched;
  *    a rejected call returns BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED and
