@@ -3,7 +3,8 @@ the benchmark times.  Selection masks are compared in full (bit-exact outside th
 tie band); attention outputs in full for the tiny and CogVideoX-2B shapes and on a
 fixed sample of query blocks ({0, 1, Qb/2, Qb-1} plus seeded random blocks,
 including the ragged last block) for the N = 75600 and N = 118800 shapes, whose
-full fp64 oracle would take hours."""
+full fp64 oracle would take hours.  The host-buffer call the benchmark's end-to-end
+figure times is compared byte for byte with the device call at Wan2.1-14B size."""
 import functools
 
 import numpy as np
@@ -115,3 +116,16 @@ def test_wan13b_fused_cdf09():
     assert bad == 0
     agree = np.all(mask.cpu().numpy() == mref, axis=-1)
     _check_rows(out, wl, qkv_cpu, mref, agree, range(wl.H), 3, seed=90)
+
+
+def test_wan14b_host_buffer_call_matches_device_call():
+    """The end-to-end call the benchmark times (pinned host buffers, default head
+    chunking) writes exactly the bytes of the device call at full Wan2.1-14B size;
+    the device call itself is checked against the oracle above."""
+    wl, (q, k, v), (qd, kd, vd) = _inputs("wan14b")
+    ref = bsa.sparse_attn_topk(qd, kd, vd, 0.5)
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    ws = bsa.make_workspace(wl.B, wl.H, wl.N, wl.d)
+    out = bsa.sparse_attn_topk_host(qp, kp, vp, 0.5, workspace=ws)
+    bsa.last_device_status(ws)
+    assert torch.equal(out, ref.cpu())
