@@ -494,3 +494,26 @@ def test_kept_mass_is_one_for_dense_and_below_one_for_sparse():
     half = ones.copy(); half[..., 1::2] = 0
     km = O.kept_mass(q, k, half, 0, 0, [0, 1, 2])
     assert np.all(km < 1) and np.all(km > 0)
+
+
+def test_kept_mass_hand_worked():
+    """d = 1 and N = 130 (query blocks of 128 and 2 rows; key blocks of 64, 64 and 2
+    keys).  k is ln 3 on keys 0-63, 0 on keys 64-127 and ln 5 on keys 128-129, so a
+    row with q = 1 gives each key weight 3, 1 or 5 (total 64*3 + 64*1 + 2*5 = 266)
+    and a row with q = 2 weights 9, 1 or 25 (total 576 + 64 + 50 = 690)."""
+    N = 130
+    k = np.zeros((1, 1, N, 1))
+    k[0, 0, :64, 0] = math.log(3.0)
+    k[0, 0, 128:, 0] = math.log(5.0)
+    q = np.ones((1, 1, N, 1))
+    q[0, 0, 128:, 0] = 2.0
+    mask = np.array([[[[1, 0, 1], [1, 1, 0]]]], dtype=np.uint8)
+    km = O.kept_mass(q, k, mask, 0, 0, [0, 1])
+    assert km.shape == (130,)
+    np.testing.assert_allclose(km[:128], 202.0 / 266.0, rtol=1e-13)
+    np.testing.assert_allclose(km[128:], 640.0 / 690.0, rtol=1e-13)
+    # the listed blocks select the rows: block 1 alone gives its two rows only
+    np.testing.assert_allclose(O.kept_mass(q, k, mask, 0, 0, [1]), 640.0 / 690.0, rtol=1e-13)
+    # and the mask row of each block is its own
+    swapped = mask[:, :, ::-1].copy()
+    np.testing.assert_allclose(O.kept_mass(q, k, swapped, 0, 0, [0])[0], 256.0 / 266.0, rtol=1e-13)

@@ -9,7 +9,7 @@ import torch
 import block_sparse_attention_14_b200 as bsa
 from block_sparse_attention_14_b200 import workloads as W
 from oracle import bsa_oracle as O
-from tests.parity import assert_close, compare_masks
+from tests.parity import assert_close
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu
@@ -68,15 +68,11 @@ def test_tiny_workload_fused_topk(cuda_device):
     q, k, v = W.make_qkv(wl)
     out, mask = bsa.sparse_attn_topk(*_cuda(q, k, v), topk=0.5, return_mask=True)
     torch.cuda.synchronize()
-    mref, P = O.select(q, k, 0.5)
-    kk = O.keep_count(0.5, wl.Kb)
-    bad, n_ex, _ = compare_masks(mask, mref, P, kk)
-    assert bad == 0
-    ref = O.block_sparse_attention(q, k, v, mref)
-    same = np.all(mask.cpu().numpy() == mref, axis=-1)  # compare rows whose masks agree
-    got = out.float().cpu().numpy()
-    rows = np.repeat(same, 128, axis=2)[:, :, :wl.N]
-    assert_close(got[rows], ref[rows], "tiny fused")
+    mref, Pr = O.select(q, k, 0.5)
+    mc = P.check_topk_mask(mask, mref, Pr, 0.5, what="tiny")
+    # every row, against the oracle's attention over the validated GPU mask
+    ref = O.block_sparse_attention(q, k, v, mc.mask)
+    assert_close(out.float().cpu().numpy(), ref, f"tiny fused; {mc}")
 
 
 @pytest.mark.parametrize("N,d,topk", [(3000, 128, 0.3), (3000, 64, 0.5), (777, 128, 0.2),
@@ -86,13 +82,10 @@ def test_fused_topk_matches_oracle(N, d, topk, cuda_device):
     q, k, v = W.make_qkv(wl)
     out, mask = bsa.sparse_attn_topk(*_cuda(q, k, v), topk=topk, return_mask=True)
     torch.cuda.synchronize()
-    mref, P = O.select(q, k, topk)
-    bad, _, diff_ex = compare_masks(mask, mref, P, O.keep_count(topk, wl.Kb))
-    assert bad == 0
-    ref = O.block_sparse_attention(q, k, v, mref)
-    same = np.all(mask.cpu().numpy() == mref, axis=-1)
-    rows = np.repeat(same, 128, axis=2)[:, :, :N]
-    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"fused {N,d,topk}")
+    mref, Pr = O.select(q, k, topk)
+    mc = P.check_topk_mask(mask, mref, Pr, topk, what=f"fused {N,d,topk}")
+    ref = O.block_sparse_attention(q, k, v, mc.mask)
+    assert_close(out.float().cpu().numpy(), ref, f"fused {N,d,topk}; {mc}")
 
 
 def test_select_equals_fused_mask_and_block_scores(cuda_device):
@@ -201,28 +194,16 @@ def test_causal_fused_topk_matches_oracle(N, d, topk, cuda_device):
     m2 = bsa.sparse_attn_select(qc, kc, topk, is_causal=True)
     torch.cuda.synchronize()
     assert torch.equal(mask, m2)
-    mref, P = O.select(q, k, topk, causal=True)
-    mg = mask.cpu().numpy()
-    Qb, Kb = wl.Qb, wl.Kb
-    for i in range(Qb):  # per-row k and eligibility; rows may differ only within the tie band
-        E = O.causal_block_limit(i, Kb)
-        kk = O.keep_count(topk, E)
-        assert np.all(mg[:, :, i, E:] == 0)
-        assert np.all(mg[:, :, i].sum(-1) == kk)
-        diff = np.any(mg[:, :, i] != mref[:, :, i], axis=-1)
-        ex = O.tie_exempt_rows(P[:, :, i:i + 1, :E], kk)[:, :, 0]
-        assert not np.any(diff & ~ex)
-    ref = O.block_sparse_attention(q, k, v, mref, causal=True)
-    same = np.all(mg == mref, axis=-1)
-    rows = np.repeat(same, 128, axis=2)[:, :, :N]
-    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"causal topk {N,d,topk}")
+    mref, Pr = O.select(q, k, topk, causal=True)
+    # per-row k over the eligible blocks; rows may differ only within the tie band
+    mc = P.check_topk_mask(mask, mref, Pr, topk, causal=True, what=f"causal topk {N,d,topk}")
+    ref = O.block_sparse_attention(q, k, v, mc.mask, causal=True)
+    assert_close(out.float().cpu().numpy(), ref, f"causal topk {N,d,topk}; {mc}")
 
 
 @pytest.mark.parametrize("N,d,tau", [(3000, 128, 0.5), (3000, 128, 0.9), (2500, 64, 0.95), (777, 128, 0.3),
                                      (4096, 64, 1.0)])
 def test_cdf_selection_and_attention_match_oracle(N, d, tau, cuda_device):
-    from tests.parity import compare_cdf_masks
-
     wl = W.custom("cdf", B=1, H=3, d=d, N=N, seed=N + 1)
     q, k, v = W.make_qkv(wl)
     qc, kc, vc = _cuda(q, k, v)
@@ -230,13 +211,10 @@ def test_cdf_selection_and_attention_match_oracle(N, d, tau, cuda_device):
     out, m2 = bsa.sparse_attn_cdf(qc, kc, vc, tau, return_mask=True)
     torch.cuda.synchronize()
     assert torch.equal(m1, m2)
-    mref, P = O.select_cdf(q, k, tau)
-    bad, _ = compare_cdf_masks(m1, mref, P, tau)
-    assert bad == 0
-    ref = O.block_sparse_attention(q, k, v, mref)
-    same = np.all(m1.cpu().numpy() == mref, axis=-1)
-    rows = np.repeat(same, 128, axis=2)[:, :, :N]
-    assert_close(out.float().cpu().numpy()[rows], ref[rows], f"cdf {N,d,tau}")
+    mref, Pr = O.select_cdf(q, k, tau)
+    mc = P.check_cdf_mask(m1, mref, Pr, tau, what=f"cdf {N,d,tau}")
+    ref = O.block_sparse_attention(q, k, v, mc.mask)
+    assert_close(out.float().cpu().numpy(), ref, f"cdf {N,d,tau}; {mc}")
 
 
 @pytest.mark.parametrize("N,d,scale,causal,order", [(3000, 128, 4.0, False, "ascending"),

@@ -2,7 +2,8 @@
 blocks, the top of the int16 index range and of the row kernels' shared-memory
 sizing) and one below it (a ragged last block): selection in full against the
 fp64 oracle, attention on sampled query blocks (the first, second, middle and
-last, plus seeded random ones)."""
+last, plus seeded random ones, and every block whose GPU mask differs from the
+oracle's inside the tie band)."""
 import numpy as np
 import pytest
 import torch
@@ -10,22 +11,22 @@ import torch
 import block_sparse_attention_14_b200 as bsa
 from block_sparse_attention_14_b200 import workloads as W
 from oracle import bsa_oracle as O
-from tests.parity import assert_close, compare_cdf_masks, compare_masks, sampled_blocks
+from tests import parity as P
+from tests.parity import assert_close, sampled_blocks
 
 pytestmark = pytest.mark.gpu
 
 
-def _rows(out, q, k, v, mask_ref, agree, blocks, N, causal=False):
+def _rows(out, q, k, v, mc, mask_ref, blocks, N, causal=False):
+    """GPU and oracle rows of the sampled query blocks plus every block whose GPU
+    mask differs from the oracle's; the oracle attends over the validated GPU mask."""
     got, ref = [], []
     o = out.cpu()
     qh, kh, vh = O.to_f64(q[0, 0]), O.to_f64(k[0, 0]), O.to_f64(v[0, 0])
-    for i in blocks:
-        if not agree[0, 0, i]:
-            continue
+    for i in sorted(set(blocks) | set(P.differing_blocks(mc, mask_ref, 0, 0))):
         lo, hi = 128 * i, min(N, 128 * i + 128)
-        ref.append(O.attention_rows(qh, kh, vh, mask_ref[0, 0, i], i, causal=causal))
+        ref.append(O.attention_rows(qh, kh, vh, mc.mask[0, 0, i], i, causal=causal))
         got.append(o[0, 0, lo:hi].float().numpy())
-    assert got, "no sampled block to compare"
     return np.concatenate(got), np.concatenate(ref)
 
 
@@ -36,12 +37,10 @@ def test_topk_at_max_length(N, d, topk, cuda_device):
     assert wl.Kb == 2048
     out, mask = bsa.sparse_attn_topk(q.cuda(), k.cuda(), v.cuda(), topk, return_mask=True)
     torch.cuda.synchronize()
-    mref, P = O.select(q, k, topk)
-    bad, _, _ = compare_masks(mask, mref, P, O.keep_count(topk, wl.Kb))
-    assert bad == 0
-    agree = np.all(mask.cpu().numpy() == mref, axis=-1)
-    got, ref = _rows(out, q, k, v, mref, agree, sampled_blocks(wl.Qb, 4, seed=N), N)
-    assert_close(got, ref, f"max-length topk {N, d}")
+    mref, Pr = O.select(q, k, topk)
+    mc = P.check_topk_mask(mask, mref, Pr, topk, what=f"max-length topk {N, d}")
+    got, ref = _rows(out, q, k, v, mc, mref, sampled_blocks(wl.Qb, 4, seed=N), N)
+    assert_close(got, ref, f"max-length topk {N, d}; {mc}")
 
 
 def test_cdf_at_max_length(cuda_device):
@@ -50,12 +49,10 @@ def test_cdf_at_max_length(cuda_device):
     q, k, v = W.make_qkv(wl)
     out, mask = bsa.sparse_attn_cdf(q.cuda(), k.cuda(), v.cuda(), tau, return_mask=True)
     torch.cuda.synchronize()
-    mref, P = O.select_cdf(q, k, tau)
-    bad, _ = compare_cdf_masks(mask, mref, P, tau)
-    assert bad == 0
-    agree = np.all(mask.cpu().numpy() == mref, axis=-1)
-    got, ref = _rows(out, q, k, v, mref, agree, sampled_blocks(wl.Qb, 4, seed=5), N)
-    assert_close(got, ref, "max-length cdf")
+    mref, Pr = O.select_cdf(q, k, tau)
+    mc = P.check_cdf_mask(mask, mref, Pr, tau, what="max-length cdf")
+    got, ref = _rows(out, q, k, v, mc, mref, sampled_blocks(wl.Qb, 4, seed=5), N)
+    assert_close(got, ref, f"max-length cdf; {mc}")
 
 
 def test_causal_topk_at_max_length(cuda_device):
@@ -64,17 +61,10 @@ def test_causal_topk_at_max_length(cuda_device):
     q, k, v = W.make_qkv(wl)
     out, mask = bsa.sparse_attn_topk(q.cuda(), k.cuda(), v.cuda(), topk, is_causal=True, return_mask=True)
     torch.cuda.synchronize()
-    mref, P = O.select(q, k, topk, causal=True)
-    mg = mask.cpu().numpy()
-    for i in range(wl.Qb):
-        E = O.causal_block_limit(i, wl.Kb)
-        kk = O.keep_count(topk, E)
-        assert np.all(mg[0, 0, i, E:] == 0) and mg[0, 0, i].sum() == kk
-        if np.any(mg[0, 0, i] != mref[0, 0, i]):
-            assert O.tie_exempt_rows(P[:, :, i:i + 1, :E], kk)[0, 0, 0]
-    agree = np.all(mg == mref, axis=-1)
-    got, ref = _rows(out, q, k, v, mref, agree, sampled_blocks(wl.Qb, 4, seed=9), N, causal=True)
-    assert_close(got, ref, "max-length causal topk")
+    mref, Pr = O.select(q, k, topk, causal=True)
+    mc = P.check_topk_mask(mask, mref, Pr, topk, causal=True, what="max-length causal topk")
+    got, ref = _rows(out, q, k, v, mc, mref, sampled_blocks(wl.Qb, 4, seed=9), N, causal=True)
+    assert_close(got, ref, f"max-length causal topk; {mc}")
 
 
 def test_host_call_at_max_length(cuda_device):
