@@ -20,6 +20,12 @@ API, after "SpargeAttention Documentation":
 * ``sparse_attn_block_scores(q, k)`` -- the compressed block-score map.
 
 q, k, v are CUDA bf16 tensors of shape [B, H, N, d] (d = 64 or 128).
+
+Every call is asynchronous on the current CUDA stream.  The kernels' waits are
+bounded; a call whose wait ran out leaves some output rows unwritten, which the
+library reports only through its device status word.  ``check=True`` reads that
+word after the call (synchronising the stream) and raises ``BsaError`` with
+status BSA_ERR_TIMEOUT; ``last_device_status(workspace)`` does the same later.
 """
 from __future__ import annotations
 
@@ -31,7 +37,8 @@ import torch
 __all__ = [
     "BsaError", "sparse_attn_topk", "block_sparse_attn_fwd", "sparse_attn_select",
     "sparse_attn_block_scores", "sparse_attn_select_cdf", "sparse_attn_cdf", "workspace_bytes", "make_workspace", "last_device_status",
-    "set_wait_timeout_ns", "token_permutation", "permute_tokens", "block_sparse_attn_plan", "block_sparse_attn_apply", "block_counts", "keep_count", "library_path", "lib",
+    "set_wait_timeout_ns", "token_permutation", "permute_tokens", "block_sparse_attn_plan", "block_sparse_attn_apply",
+    "sparse_attn_topk_host", "sparse_attn_topk_noalloc", "noalloc_status", "block_counts", "library_path", "lib",
 ]
 
 BLOCK_Q = 128
@@ -100,6 +107,10 @@ def lib() -> ctypes.CDLL:
         L.bsa_last_device_status.argtypes = [vp, vp]
         L.bsa_set_wait_timeout_ns.restype = None
         L.bsa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.sparse_attn_topk_noalloc.restype = i32
+        L.sparse_attn_topk_noalloc.argtypes = [vp, vp, vp, Shape, f32, i32, vp, vp, vp]
+        L.sparse_attn_topk_noalloc_status.restype = i32
+        L.sparse_attn_topk_noalloc_status.argtypes = [vp]
         _LIB = L
     return _LIB
 
@@ -111,15 +122,6 @@ def _check(status: int) -> None:
 
 def block_counts(N: int) -> tuple[int, int]:
     return -(-N // BLOCK_Q), -(-N // BLOCK_K)
-
-
-def keep_count(topk: float, Kb: int) -> int:
-    """Kept key blocks per query block, as the library computes it (ceil, clamped)."""
-    import math
-    import struct
-
-    t = struct.unpack("f", struct.pack("f", topk))[0]
-    return max(1, min(Kb, math.ceil(t * Kb)))
 
 
 def _shape_of(q: torch.Tensor) -> Shape:
@@ -180,8 +182,13 @@ def _mask_arg(mask: torch.Tensor, q: torch.Tensor) -> torch.Tensor:
     return mask
 
 
+def _checked(ws, check: bool) -> None:
+    if check:
+        last_device_status(ws)
+
+
 def sparse_attn_topk(q, k, v, topk: float = 0.5, is_causal: bool = False, *, out=None,
-                     return_mask: bool = False, workspace=None):
+                     return_mask: bool = False, workspace=None, check: bool = False):
     """Top-k block selection followed by block-sparse attention.
 
     Returns out (bf16 [B, H, N, d]), or (out, mask) with return_mask=True.
@@ -195,12 +202,13 @@ def sparse_attn_topk(q, k, v, topk: float = 0.5, is_causal: bool = False, *, out
     _check(lib().sparse_attn_topk(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q), float(topk),
                                   int(bool(is_causal)), out.data_ptr(),
                                   mask.data_ptr() if mask is not None else None, wp, wn, _stream(q)))
+    _checked(ws, check)
     return (out, mask) if return_mask else out
 
 
 def sparse_attn_topk_host(q_host, k_host, v_host, topk: float = 0.5, is_causal: bool = False, *,
                           out_host=None, device_buffers=None, workspace=None, chunks: int = 0,
-                          device="cuda"):
+                          device="cuda", check: bool = False):
     """sparse_attn_topk on pinned host tensors, with the host<->device copies
     pipelined over chunks of heads.  device_buffers: (q, k, v, out) device tensors
     of the same shape (allocated if None).  Runs on the current stream of
@@ -223,10 +231,12 @@ def sparse_attn_topk_host(q_host, k_host, v_host, topk: float = 0.5, is_causal: 
                                        out_host.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
                                        od.data_ptr(), wp, wn, int(chunks), _stream(qd)))
     torch.cuda.current_stream(qd.device).synchronize()
+    _checked(ws, check)
     return out_host
 
 
-def block_sparse_attn_fwd(q, k, v, mask_id=None, is_causal: bool = False, *, out=None, workspace=None):
+def block_sparse_attn_fwd(q, k, v, mask_id=None, is_causal: bool = False, *, out=None, workspace=None,
+                          check: bool = False):
     """Attention over the kept 128 x 64 tiles of mask_id ([B, H, ceil(N/128), ceil(N/64)],
     nonzero = keep; None = dense)."""
     _qkv(q, k, v)
@@ -237,6 +247,7 @@ def block_sparse_attn_fwd(q, k, v, mask_id=None, is_causal: bool = False, *, out
     _check(lib().block_sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q),
                                        m.data_ptr() if m is not None else None, int(bool(is_causal)),
                                        out.data_ptr(), wp, wn, _stream(q)))
+    _checked(ws, check)
     return out
 
 
@@ -270,7 +281,7 @@ def sparse_attn_select_cdf(q, k, threshold: float, *, mask_out=None, workspace=N
 
 
 def sparse_attn_cdf(q, k, v, threshold: float = 0.9, is_causal: bool = False, *, out=None,
-                    return_mask: bool = False, workspace=None):
+                    return_mask: bool = False, workspace=None, check: bool = False):
     """cdfthreshd selection followed by block-sparse attention."""
     _qkv(q, k, v)
     out = torch.empty_like(q) if out is None else out
@@ -281,6 +292,7 @@ def sparse_attn_cdf(q, k, v, threshold: float = 0.9, is_causal: bool = False, *,
     _check(lib().sparse_attn_cdf(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q), float(threshold),
                                  int(bool(is_causal)), out.data_ptr(),
                                  mask.data_ptr() if mask is not None else None, wp, wn, _stream(q)))
+    _checked(ws, check)
     return (out, mask) if return_mask else out
 
 
@@ -308,7 +320,7 @@ def block_sparse_attn_plan(q, mask_id=None, is_causal: bool = False, *, workspac
     return ws
 
 
-def block_sparse_attn_apply(q, k, v, workspace, is_causal: bool = False, *, out=None):
+def block_sparse_attn_apply(q, k, v, workspace, is_causal: bool = False, *, out=None, check: bool = False):
     """Attention over the plan held in `workspace` (from sparse_attn_select,
     sparse_attn_topk or block_sparse_attn_plan on the same shape)."""
     _qkv(q, k, v)
@@ -317,6 +329,7 @@ def block_sparse_attn_apply(q, k, v, workspace, is_causal: bool = False, *, out=
     _check(lib().block_sparse_attn_apply(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q),
                                          int(bool(is_causal)), out.data_ptr(), workspace.data_ptr(),
                                          workspace.numel(), _stream(q)))
+    _checked(workspace, check)
     return out
 
 
@@ -344,10 +357,38 @@ def permute_tokens(x: torch.Tensor, perm: torch.Tensor, inverse: bool = False, *
     return out
 
 
+def sparse_attn_topk_noalloc(q, k, v, topk: float = 0.5, is_causal: bool = False, *, out=None,
+                             return_mask: bool = False, check: bool = False):
+    """sparse_attn_topk with the library's static device scratch in place of a
+    workspace, for callers that cannot allocate device memory for one (only
+    `out` and the optional mask are allocated here, unless passed in).  Calls on
+    one device share the scratch: order them on one stream."""
+    _qkv(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    _qkv(q, out)
+    B, H, N, _ = q.shape
+    mask = torch.empty(B, H, *block_counts(N), dtype=torch.uint8, device=q.device) if return_mask else None
+    _check(lib().sparse_attn_topk_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), _shape_of(q), float(topk),
+                                          int(bool(is_causal)), out.data_ptr(),
+                                          mask.data_ptr() if mask is not None else None, _stream(q)))
+    if check:
+        noalloc_status(q.device)
+    return (out, mask) if return_mask else out
+
+
+def noalloc_status(device="cuda") -> None:
+    """Synchronise and raise BsaError if the last no-allocation call on `device`
+    recorded a failure."""
+    dev = torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib().sparse_attn_topk_noalloc_status(torch.cuda.current_stream(dev).cuda_stream))
+
+
 def last_device_status(workspace: torch.Tensor) -> None:
     """Synchronise and raise BsaError if the last call on `workspace` recorded a failure."""
     _check(lib().bsa_last_device_status(workspace.data_ptr(), _stream(workspace)))
 
 
 def set_wait_timeout_ns(ns: int) -> None:
+    """Limit of the kernels' bounded waits in nanoseconds (0 restores the 10 s default)."""
     lib().bsa_set_wait_timeout_ns(int(ns))

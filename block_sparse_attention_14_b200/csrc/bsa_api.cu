@@ -16,7 +16,8 @@ namespace bsa {
 namespace {
 
 thread_local char g_last_error[512] = {0};
-std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+constexpr uint64_t kDefaultTimeoutNs = 10000000000ull;  // 10 s
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 
 bsa_status fail(bsa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 bsa_status fail(bsa_status s, const char* fmt, ...) {
@@ -83,14 +84,6 @@ bsa_status check_topk(float topk) {
   return BSA_OK;
 }
 
-int keep_count(float topk, int Kb) {
-  const double t = static_cast<double>(topk);
-  long long k = static_cast<long long>(ceil(t * static_cast<double>(Kb)));
-  if (k < 1) k = 1;
-  if (k > Kb) k = Kb;
-  return static_cast<int>(k);
-}
-
 #define BSA_TRY(x)                          \
   do {                                      \
     bsa_status _s = (x);                    \
@@ -141,6 +134,29 @@ struct PipelineResources {
 }  // namespace
 
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+
+int keep_count(float topk, int Kb) {
+  const double t = static_cast<double>(topk);
+  long long k = static_cast<long long>(ceil(t * static_cast<double>(Kb)));
+  if (k < 1) k = 1;
+  if (k > Kb) k = Kb;
+  return static_cast<int>(k);
+}
+
+int max_score_heads(int B, int H, int N, int d, size_t capacity) {
+  const size_t one = workspace_layout(B, H, N, d, nullptr, nullptr, 1);
+  if (one > capacity) return 0;
+  const size_t Qb = (static_cast<size_t>(N) + kBlockQ - 1) / kBlockQ;
+  const size_t Kb = (static_cast<size_t>(N) + kBlockK - 1) / kBlockK;
+  const size_t per_head = Qb * padded_kb(static_cast<int>(Kb)) * sizeof(float);
+  // Every section is rounded up to 256 bytes, so the layout with SH heads is the
+  // layout without the score section plus SH * per_head rounded up to 256.
+  const size_t fixed = one - align256(per_head);
+  const size_t BH = static_cast<size_t>(B) * H;
+  size_t sh = (capacity - fixed) / per_head;
+  if (sh > BH) sh = BH;
+  return static_cast<int>(sh);
+}
 
 void set_last_error(const char* msg) {
   snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
@@ -193,7 +209,9 @@ const char* bsa_status_string(bsa_status s) {
 
 const char* bsa_last_error_message(void) { return g_last_error; }
 
-void bsa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns < 1000 ? 1000 : ns); }
+void bsa_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : (ns < 1000 ? 1000 : ns));
+}
 
 size_t bsa_workspace_bytes(bsa_shape s) {
   if (check_shape(s) != BSA_OK) return 0;

@@ -32,6 +32,15 @@ inline int padded_kb(int Kb) { return (Kb + 3) & ~3; }
 // Current limit of the kernels' bounded waits (bsa_set_wait_timeout_ns).
 uint64_t wait_timeout_ns();
 
+// Kept key blocks per row for a top-k fraction: clamp(ceil(topk * Kb), 1, Kb),
+// in double precision on the float value of topk.
+int keep_count(float topk, int Kb);
+
+// The largest number of heads whose block-score matrices fit, together with the
+// rest of the workspace layout, in `capacity` bytes (at most B*H; 0 if not even
+// one head fits).
+int max_score_heads(int B, int H, int N, int d, size_t capacity);
+
 // Records the message returned by bsa_last_error_message() on this thread.
 void set_last_error(const char* msg);
 

@@ -1,7 +1,9 @@
 // sparse_attn_topk_noalloc: the fused selection + attention call for callers
-// that cannot allocate device memory.  Its scratch (pooled means, kept-block
-// lists, status word) lives in a file-scope __device__ array instead of a
-// caller-provided workspace; the caller still passes q, k, v, out and mask.
+// that cannot allocate device memory.  Its scratch (pooled means, block
+// scores, kept-block lists, status word) lives in a file-scope __device__ array
+// instead of a caller-provided workspace; the caller still passes q, k, v, out
+// and the optional mask.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -20,25 +22,59 @@ constexpr size_t kStaticScratchBytes = 32ull << 20;
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 256;
+struct ScratchEntry {
+  void* ctx;  // CUDA context the address was looked up in
+  void* ptr;  // device address of that context's copy of g_static_scratch
+};
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of this device's copy of g_static_scratch.  In host code the
-// symbol's name is only a host-side handle, so the address is looked up once
-// per device (with that device current) and cached.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the current device's copy of g_static_scratch.  In host
+// code the symbol's name is only a host-side handle, so the address is looked
+// up with cudaGetSymbolAddress (with the device current) and cached per device
+// and CUDA context: a new context on the device (after cudaDeviceReset, say)
+// reloads the module, so its address is looked up afresh.
 cudaError_t scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (get == nullptr) return cudaErrorInitializationError;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
+  if (ctx == nullptr) {
+    // No context is current on this thread yet: the symbol lookup initialises
+    // the device's primary context (and loads the module), then it is current.
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_static_scratch)) != cudaSuccess) return e;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorInitializationError;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchEntry& s = g_scratch[dev];
+  if (s.ptr == nullptr || s.ctx != static_cast<void*>(ctx)) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    s.ptr = p;
+    s.ctx = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = s.ptr;
   return cudaSuccess;
 }
 
@@ -59,7 +95,6 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
   if (s.B < 1 || s.H < 1 || s.N < 1 || (s.d != 64 && s.d != 128) || s.N > kBlockK * kMaxKb ||
       static_cast<int64_t>(s.B) * s.H > 65535)
     return reject(BSA_ERR_INVALID_ARG, "bad shape: need B, H, N >= 1, d in {64, 128}, N <= 131072, B*H <= 65535");
-  if (is_causal != 0) return reject(BSA_ERR_UNSUPPORTED, "is_causal != 0 is not supported");
   const void* ptrs[4] = {q, k, v, out};
   for (const void* p : ptrs)
     if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) != 0)
@@ -85,30 +120,34 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
              need, kStaticScratchBytes);
     return reject(BSA_ERR_INVALID_ARG, msg);
   }
-  const int BHs = s.B * s.H;
-  int score_heads = 1;
-  while (score_heads < BHs &&
-         workspace_layout(s.B, s.H, s.N, s.d, nullptr, nullptr, 2 * score_heads) <= kStaticScratchBytes)
-    score_heads *= 2;
+  const int BH = s.B * s.H;
+  const int score_heads = max_score_heads(s.B, s.H, s.N, s.d, kStaticScratchBytes);
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   Workspace w;
   workspace_layout(s.B, s.H, s.N, s.d, &w, base, score_heads);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int BH = s.B * s.H;
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
-  long long kk = static_cast<long long>(ceil(static_cast<double>(topk) * static_cast<double>(Kb)));
-  kk = kk < 1 ? 1 : (kk > Kb ? Kb : kk);
+  const int causal = is_causal != 0;
   // The status word must start at zero; everything else is overwritten.
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
       (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
-      (e = launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, static_cast<int>(kk), topk, 0, mask_out, w.idx,
-                         w.cnt, st)) != cudaSuccess)
+      (e = launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk,
+                         causal, mask_out, w.idx, w.cnt, st)) != cudaSuccess)
     return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   const char* why = nullptr;
-  e = launch_attention(q, k, v, out, BH, s.N, s.d, 0, w.idx, w.cnt, w.status, wait_timeout_ns(), st,
+  e = launch_attention(q, k, v, out, BH, s.N, s.d, causal, w.idx, w.cnt, w.status, wait_timeout_ns(), st,
                        &why);
   if (e != cudaSuccess) return reject(BSA_ERR_CUDA, why ? why : cudaGetErrorString(e));
   return BSA_OK;
+}
+
+extern "C" bsa_status sparse_attn_topk_noalloc_status(void* stream) {
+  set_last_error("");
+  void* base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess) return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
+  // The status word sits at the start of the scratch, as in a caller workspace.
+  return bsa_last_device_status(base, stream);
 }

@@ -58,8 +58,7 @@ extern "C" {
 typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment, topk or workspace size */
-  BSA_ERR_UNSUPPORTED = 2, /* an unsupported mode combination (is_causal with cdfthreshd or the
-                              no-allocation call) */
+  BSA_ERR_UNSUPPORTED = 2, /* an unsupported mode combination (is_causal with cdfthreshd) */
   BSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   BSA_ERR_TIMEOUT = 4      /* a bounded wait inside a kernel ran out */
 } bsa_status;
@@ -161,10 +160,10 @@ bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, 
                                    void* stream);
 
 /* No-allocation variant of sparse_attn_topk (same arguments minus the
- * workspace; same kernels, same results).  The pages have no counterpart: this
- * call exists for callers that cannot allocate device memory, such as a
- * serving engine that reserves all free device memory for its own pool at
- * start-up (so no memory is left for a workspace), or a caller on a
+ * workspace, is_causal included; same kernels, same results).  The pages have
+ * no counterpart: this call exists for callers that cannot allocate device
+ * memory, such as a serving engine that reserves all free device memory for its
+ * own pool at start-up (so no memory is left for a workspace), or a caller on a
  * latency-critical path that must not trigger the device-wide synchronisation
  * of cudaFree.  Its scratch is a file-scope device array of 32 MiB, held on
  * every GPU that loads the library until the process exits.  The scratch holds
@@ -173,14 +172,22 @@ bsa_status block_sparse_attn_apply(const void* q, const void* k, const void* v, 
  * workspace with one head's score matrix exceeds 32 MiB are rejected with
  * BSA_ERR_INVALID_ARG before anything is launched.  The first call on a device
  * looks up that device's copy of the array with cudaGetSymbolAddress (with the
- * device current), so make the first call on each device before any stream
- * capture.  Every call on a device shares the one array: calls that may
- * overlap on the GPU (different streams, other threads) race and corrupt each
- * other's results, so order them on one stream.  The call allocates nothing.
- * mask_out is optional (NULL: not written). */
+ * device current) and caches it per device and CUDA context (a new context,
+ * after cudaDeviceReset for example, is looked up afresh), so make the first
+ * call on each device, and the first after a reset, before any stream capture.
+ * Every call on a device shares the one array, which keeps the last call's
+ * contents: calls that may overlap on the GPU (different streams, other
+ * threads) race and corrupt each other's results, so order them on one stream.
+ * The call allocates nothing.  mask_out is optional (NULL: not written). */
 bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, const void* v, bsa_shape s,
                                     float topk, int is_causal, void* out, uint8_t* mask_out,
                                     void* stream);
+
+/* Status of the last sparse_attn_topk_noalloc call on the current device, as
+ * bsa_last_device_status reports it for a workspace: synchronises `stream`, then
+ * returns BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out and some output rows
+ * were left unwritten) or BSA_ERR_CUDA.  No counterpart on the pages. */
+bsa_status sparse_attn_topk_noalloc_status(void* stream);
 
 /* sparse_attn_topk on HOST buffers, pipelined over chunks of heads: while the
  * attention of chunk c runs, chunk c+1's q/k/v are copied in on one internal
@@ -238,11 +245,18 @@ bsa_status bsa_permute_tokens(const void* src, void* dst, bsa_shape s, const int
 
 /* Synchronises `stream`, then reports what the kernels of the last call that
  * used `ws` recorded: BSA_OK, BSA_ERR_TIMEOUT (a bounded wait ran out), or
- * BSA_ERR_CUDA if the stream holds an error. */
+ * BSA_ERR_CUDA if the stream holds an error.  A call whose wait ran out returns
+ * BSA_OK itself (it only launches) and leaves some output rows unwritten, so a
+ * caller that must know checks here after the call. */
 bsa_status bsa_last_device_status(const void* ws, void* stream);
 
 /* Limit of every bounded wait inside the kernels, in nanoseconds (process-wide;
- * default 2e9).  Values below 1000 are raised to 1000. */
+ * default 1e10, i.e. 10 s; 0 restores the default; other values below 1000 are
+ * raised to 1000).  The limit is measured on the GPU's global timer, which keeps
+ * running while the context is time-sliced out by other work on a shared GPU,
+ * so it is set far above any call's own duration (a CTA's longest wait is a few
+ * microseconds in a healthy run); a lower limit risks reporting a timeout for a
+ * call that was only preempted. */
 void bsa_set_wait_timeout_ns(uint64_t ns);
 
 #ifdef __cplusplus
