@@ -5,15 +5,24 @@ One step = one pass of the whole path on the Wan2.1-14B-shaped self-attention
 call (B=1, H=40, N=75600 = 21x45x80 tokens, d=128, bf16, topk=0.5): mean
 pooling, block scores + top-k selection, and block-sparse attention over the
 kept 128x64 tiles.  The timed step issues sparse_attn_select and then
-block_sparse_attn_apply on one stream -- the same three kernels, in the same
-order, that the fused sparse_attn_topk call launches -- so that the attention
-kernel can be timed on its own with CUDA events; the fused call is timed too.
+block_sparse_attn_apply on one stream -- the same kernels, in the same order,
+that the fused sparse_attn_topk call launches -- so that the attention kernel
+can be timed on its own with CUDA events; the fused call is timed too.
 
 Prints one JSON line (rank 0).  Metric: dense-equivalent TFLOPS
 (4*B*H*N^2*d / step time), plus ms/call and the fraction of the measured bf16
 tensor-core peak reached by the attention kernel on its kept tiles.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {b200,reference}]
+                    [--workload W] [--call {topk,mask,cdf}] [--topk T] [--density P]
+                    [--threshold C] [--causal] [--plan-reuse R] [--sweep]
+
+--call mask times a caller-supplied random block mask at --density (compaction
+then attention, or block_sparse_attn_fwd fused); --call cdf the cdfthreshd
+selection at --threshold; --causal the causal variant; --plan-reuse R one
+selection followed by R applies of its plan (the AB-Attention refresh pattern),
+reporting the amortised time per call.  --sweep prints one line per row of the
+workload table (every config and mode), without the CPU and end-to-end legs.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
 call (weak scaling, no collective on the data path); the step time is the
@@ -60,7 +69,14 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--workload", default="wan14b", choices=sorted(W.WORKLOADS))
+    p.add_argument("--call", choices=["topk", "mask", "cdf"], default="topk")
     p.add_argument("--topk", type=float, default=0.5)
+    p.add_argument("--density", type=float, default=0.5, help="caller-mask density (--call mask)")
+    p.add_argument("--threshold", type=float, default=0.9, help="cdfthreshd threshold (--call cdf)")
+    p.add_argument("--causal", action="store_true")
+    p.add_argument("--plan-reuse", type=int, default=1,
+                   help="applies of each selection's plan per step (amortised per call)")
+    p.add_argument("--sweep", action="store_true", help="one line per row of the workload table")
     p.add_argument("--heads", type=int, default=0,
                    help="override H (small profiling case only; not a bench line)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -236,6 +252,10 @@ def blas_threads() -> int:
 
 
 def run_reference(args, world, rank):
+    """The oracle, as it stands, on a bounded sample of the bench's workload.  Each
+    timed step runs the sample (one head's selection plus attention for some of
+    its query blocks); the line's value is the extrapolation of that sample to
+    the full call, flagged as such."""
     if rank != 0:
         return 0
     wl = W.WORKLOADS[args.workload]
@@ -252,11 +272,14 @@ def run_reference(args, world, rank):
     value = wl.dense_flops() / est / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, args.topk, wl.H),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / max(1, args.steps) * 1e3,
+        "extrapolated": True, "extrapolated_ms_per_call": est * 1e3,
+        "step_is": "one bounded sample of the call (see cpu_baseline.sample); value is that sample "
+                   "extrapolated to the full call",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl, "topk", args.topk, False, wl.H),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "extrapolated": True},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -264,14 +287,208 @@ def run_reference(args, world, rank):
     return 0
 
 
-def workload_config(wl, topk, H):
-    return {"workload": f"{wl.name}: {wl.note}", "B": wl.B, "H": H, "N": wl.N, "d": wl.d,
-            "grid_thw": list(wl.grid), "topk": topk, "call": "sparse_attn_topk (select + apply)",
-            "l2": "inputs larger than L2 (q/k/v/out 4 x %.0f MB); no flush" % (wl.B * H * wl.N * wl.d * 2 / 1e6),
-            "parallelism": "replicas (one independent call per GPU)"}
+CALL_NAMES = {"topk": "sparse_attn_select + block_sparse_attn_apply (= sparse_attn_topk)",
+              "mask": "block_sparse_attn_plan + block_sparse_attn_apply (= block_sparse_attn_fwd, caller mask)",
+              "cdf": "sparse_attn_select_cdf + block_sparse_attn_apply (= sparse_attn_cdf)"}
+
+
+def workload_config(wl, call, param, causal, H, plan_reuse=1):
+    knob = {"topk": "topk", "mask": "density", "cdf": "threshold"}[call]
+    cfg = {"workload": f"{wl.name}: {wl.note}", "B": wl.B, "H": H, "N": wl.N, "d": wl.d,
+           "grid_thw": list(wl.grid), knob: param, "causal": bool(causal), "call": CALL_NAMES[call],
+           "l2": "inputs larger than L2 (q/k/v/out 4 x %.0f MB); no flush" % (wl.B * H * wl.N * wl.d * 2 / 1e6)
+           if 4 * wl.B * H * wl.N * wl.d * 2 > 126e6 else "inputs fit in L2 (launch-bound parity case)",
+           "parallelism": "replicas (one independent call per GPU)"}
+    if plan_reuse > 1:
+        cfg["plan_reuse"] = plan_reuse
+    return cfg
+
+
+def metric_name(wl, call, param, causal, plan_reuse=1):
+    if (wl.name, call, param, causal, plan_reuse) == ("wan14b", "topk", 0.5, False, 1):
+        return METRIC
+    knob = {"topk": "topk", "mask": "caller mask p", "cdf": "cdfthreshd"}[call]
+    extra = (" causal" if causal else "") + (f" plan reused x{plan_reuse}" if plan_reuse > 1 else "")
+    return f"ms/call and dense-equiv TFLOPS, {wl.name} {knob}={param}{extra}, % of bf16 TC peak"
+
+
+def dense_flops(wl, H, causal):
+    """Dense-attention FLOPs of the call: 4 B H N^2 d, or for causal attention the
+    4 B H d N (N + 1) / 2 of the lower triangle."""
+    N = float(wl.N)
+    return 4.0 * wl.B * H * wl.d * (N * (N + 1) / 2 if causal else N * N)
 
 
 # ------------------------------------------------------------------- GPU arm
+class Case:
+    """One timed configuration: the selection-or-compaction call followed by
+    `plan_reuse` applies of its plan, on device-resident inputs."""
+
+    def __init__(self, bsa, wl, H, qkv, call, param, causal, plan_reuse=1):
+        self.bsa, self.wl, self.H = bsa, wl, H
+        self.q, self.k, self.v = qkv
+        self.call, self.param, self.causal, self.R = call, param, bool(causal), max(1, plan_reuse)
+        B, N, d = wl.B, wl.N, wl.d
+        self.out = torch.empty_like(self.q)
+        self.ws = bsa.make_workspace(B, H, N, d)
+        self.mask = torch.empty(B, H, wl.Qb, wl.Kb, dtype=torch.uint8, device="cuda")
+        if call == "mask":
+            self.mask.copy_(W.make_random_mask(W.Workload(wl.name, B=B, H=H, d=d, grid=wl.grid,
+                                                          text=wl.text, seed=wl.seed), param))
+
+    def select(self):
+        b, c = self.bsa, self.causal
+        if self.call == "topk":
+            b.sparse_attn_select(self.q, self.k, self.param, c, mask_out=self.mask, workspace=self.ws)
+        elif self.call == "cdf":
+            b.sparse_attn_select_cdf(self.q, self.k, self.param, mask_out=self.mask, workspace=self.ws)
+        else:
+            b.block_sparse_attn_plan(self.q, self.mask, c, workspace=self.ws)
+
+    def apply(self):
+        self.bsa.block_sparse_attn_apply(self.q, self.k, self.v, self.ws, self.causal, out=self.out)
+
+    def fused(self):
+        b, c = self.bsa, self.causal
+        if self.call == "topk":
+            b.sparse_attn_topk(self.q, self.k, self.v, self.param, c, out=self.out, workspace=self.ws)
+        elif self.call == "cdf":
+            b.sparse_attn_cdf(self.q, self.k, self.v, self.param, c, out=self.out, workspace=self.ws)
+        else:
+            b.block_sparse_attn_fwd(self.q, self.k, self.v, self.mask, c, out=self.out, workspace=self.ws)
+
+    def launches_per_step(self):
+        # pool + dots + row kernel for a selection, one compaction kernel for a
+        # caller mask; one attention kernel per apply
+        return (1 if self.call == "mask" else 3) + self.R
+
+    def time(self, K, Wm, world, local, fused=True):
+        stream = torch.cuda.current_stream()
+        clocks = ClockSampler(local)
+        clocks.start()
+        for _ in range(Wm):
+            self.select()
+            for _ in range(self.R):
+                self.apply()
+        self.bsa.last_device_status(self.ws)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        barrier(world)
+        torch.cuda.synchronize()
+        t_begin = time.time()
+        for i in range(K):
+            ev[i][0].record(stream)
+            self.select()
+            ev[i][1].record(stream)
+            for _ in range(self.R):
+                self.apply()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        t_end = time.time()
+        barrier(world)
+        clk = clocks.stop(t_begin, t_end)
+        self.bsa.last_device_status(self.ws)
+        step_s = ev[0][0].elapsed_time(ev[K - 1][2]) / 1e3 / K
+        sel_s = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+        attn_s = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3 / self.R
+        res = {"step_s": step_s, "call_s": step_s / self.R, "sel_s": sel_s, "attn_s": attn_s, "clocks": clk,
+               "density": float(self.mask.float().mean().item()) if not self.causal or self.call != "mask"
+               else None}
+        if self.call == "mask" and self.causal:
+            # the caller mask's entries past block 2i+1 are ignored under causal attention
+            Qb, Kb = self.wl.Qb, self.wl.Kb
+            elig = torch.arange(Kb, device="cuda")[None, :] <= 2 * torch.arange(Qb, device="cuda")[:, None] + 1
+            res["density"] = float((self.mask.bool() & elig).float().mean().item())
+        res["kept"] = int(self.mask.sum().item()) if self.call != "mask" else None
+        if fused:
+            for _ in range(2):
+                self.fused()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(K):
+                self.fused()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            self.bsa.last_device_status(self.ws)
+            res["fused_s"] = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world)
+        res["step_max_s"] = max_over_ranks(step_s, world)
+        return res
+
+
+def rooflines(case, res, peaks, kind, traffic):
+    wl, H = case.wl, case.H
+    B, N, d = wl.B, wl.N, wl.d
+    kept_flops = 4.0 * B * H * N * N * d * res["density"]
+    achieved = kept_flops / res["attn_s"] / 1e12
+    roofline = {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": traffic, "peak_kind": f"bf16 dense burst, of {kind}",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "algorithmic_flops_per_launch": kept_flops, "avg_launch_ms": res["attn_s"] * 1e3}
+    rows = B * H * wl.Qb
+    if case.call == "mask":
+        sel_bytes = rows * wl.Kb + 2 * int(case.mask.sum().item()) + 4 * rows
+        kern = "compact_kernel"
+    else:
+        sel_bytes = 2 * B * H * N * d * 2 + rows * wl.Kb + 2 * res["kept"]
+        kern = "pool_kernel + dots_kernel + " + ("select_cdf_kernel" if case.call == "cdf" else "select_kernel")
+    roofline_select = {"bound": "hbm", "kernel": kern, "achieved": sel_bytes / res["sel_s"] / 1e9,
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": sel_bytes / res["sel_s"] / 1e9 / peaks["hbm_gbs"],
+                       "algorithmic_bytes_per_call": sel_bytes, "avg_call_ms": res["sel_s"] * 1e3}
+    return roofline, kept_flops, roofline_select
+
+
+def case_line(case, res, world, K, Wm, peaks, kind, traffic):
+    wl, H = case.wl, case.H
+    dflops = dense_flops(wl, H, case.causal)
+    roofline, kept_flops, roofline_select = rooflines(case, res, peaks, kind, traffic)
+    call_max = res["step_max_s"] / case.R
+    line = {
+        "metric": metric_name(wl, case.call, case.param, case.causal, case.R),
+        "value": whole_job_value(dflops, call_max, world), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": res["step_max_s"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, case.call, case.param, case.causal, H, case.R),
+        "roofline": roofline, "roofline_select": roofline_select,
+        "gpu_launches": case.launches_per_step() * K, "clocks": res["clocks"],
+        "breakdown": {"select_ms": res["sel_s"] * 1e3, "attention_ms": res["attn_s"] * 1e3,
+                      "ms_per_call": call_max * 1e3, "fused_call_ms": res.get("fused_s", 0) * 1e3 or None,
+                      "density": res["density"], "kept_tflop": kept_flops / 1e12,
+                      "dense_tflop": dflops / 1e12},
+    }
+    if case.R > 1:
+        line["breakdown"]["plan_reuse"] = {"applies_per_selection": case.R,
+                                           "amortised_ms_per_call": call_max * 1e3,
+                                           "select_ms": res["sel_s"] * 1e3, "apply_ms": res["attn_s"] * 1e3}
+    return line
+
+
+# Rows of the workload table: (workload, call, knob value, causal, plan reuse).
+SWEEP = [
+    ("tiny", "topk", 0.5, False, 1),
+    ("cogvideox2b", "topk", 0.5, False, 1),
+    ("cogvideox2b", "topk", 0.5, True, 1),
+    ("wan13b", "topk", 1.0, False, 1),
+    ("wan13b", "topk", 0.5, False, 1),
+    ("wan13b", "topk", 0.3, False, 1),
+    ("wan13b", "topk", 0.1, False, 1),
+    ("wan13b", "cdf", 0.9, False, 1),
+    ("wan13b", "cdf", 0.5, False, 1),
+    ("wan14b", "mask", 0.5, False, 1),
+    ("wan14b", "mask", 0.1, False, 1),
+    ("wan14b", "topk", 0.5, False, 1),
+    ("wan14b", "topk", 0.5, True, 1),
+    ("wan14b", "topk", 0.5, False, 4),
+    ("hunyuan13b", "topk", 0.1, False, 1),
+]
+
+
+def knob(args):
+    return {"topk": args.topk, "mask": args.density, "cdf": args.threshold}[args.call]
+
+
 def run_b200(args, world, rank, local):
     import block_sparse_attention_14_b200 as bsa
 
@@ -282,78 +499,59 @@ def run_b200(args, world, rank, local):
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    wl = W.WORKLOADS[args.workload]
-    H = args.heads or wl.H
-    wl = W.Workload(wl.name, B=wl.B, H=H, d=wl.d, grid=wl.grid, text=wl.text, topk=wl.topk,
-                    seed=wl.seed + rank, note=wl.note)
-    q_h, k_h, v_h = W.make_qkv(wl)
-    q, k, v = q_h.cuda(), k_h.cuda(), v_h.cuda()
-    B, N, d = wl.B, wl.N, wl.d
-    out = torch.empty_like(q)
-    ws = bsa.make_workspace(B, H, N, d)
-    mask = torch.empty(B, H, wl.Qb, wl.Kb, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
+    peaks, kind = load_peaks()
     K, Wm = args.steps, args.warmup
 
-    def step():
-        bsa.sparse_attn_select(q, k, args.topk, mask_out=mask, workspace=ws)
-        bsa.block_sparse_attn_apply(q, k, v, ws, out=out)
+    def inputs(name):
+        base = W.WORKLOADS[name]
+        H = args.heads or base.H
+        wl = W.Workload(base.name, B=base.B, H=H, d=base.d, grid=base.grid, text=base.text,
+                        topk=base.topk, seed=base.seed + rank, note=base.note)
+        q_h, k_h, v_h = W.make_qkv(wl)
+        return wl, H, (q_h, k_h, v_h), (q_h.cuda(), k_h.cuda(), v_h.cuda())
 
-    clocks = ClockSampler(local)
-    clocks.start()
-    for _ in range(Wm):
-        step()
-    bsa.last_device_status(ws)
-    torch.cuda.synchronize()
+    if args.sweep:
+        cur = None
+        for name, call, param, causal, reuse in SWEEP:
+            if cur is None or cur[0].name != name:
+                cur = None
+                torch.cuda.empty_cache()
+                cur = inputs(name)
+            wl, H, _, qkv = cur
+            case = Case(bsa, wl, H, qkv, call, param, causal, reuse)
+            res = case.time(K, Wm, world, local, fused=reuse == 1)
+            traffic = recorded_traffic(wl.name) if (call, param, causal) == ("topk", 0.5, False) else None
+            line = case_line(case, res, world, K, Wm, peaks, kind, traffic)
+            line["sweep"] = True
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            del case
+        if world > 1:
+            import torch.distributed as dist
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    t_begin = time.time()
-    for i in range(K):
-        ev[i][0].record(stream)
-        bsa.sparse_attn_select(q, k, args.topk, mask_out=mask, workspace=ws)
-        ev[i][1].record(stream)
-        bsa.block_sparse_attn_apply(q, k, v, ws, out=out)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    t_end = time.time()
-    barrier(world)
-    clk = clocks.stop(t_begin, t_end)
-    bsa.last_device_status(ws)
-    step_s = ev[0][0].elapsed_time(ev[K - 1][2]) / 1e3 / K
-    sel_s = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    attn_s = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    step_max = max_over_ranks(step_s, world)
+            dist.destroy_process_group()
+        return 0
 
-    density = float(mask.float().mean().item())
-    dense_flops = wl.dense_flops()
-    kept_flops = dense_flops * density
-
-    fused_ms = None
-    if not args.no_fused:
-        for _ in range(2):
-            bsa.sparse_attn_topk(q, k, v, args.topk, out=out, workspace=ws)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(K):
-            bsa.sparse_attn_topk(q, k, v, args.topk, out=out, workspace=ws)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        fused_ms = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    wl, H, (q_h, k_h, v_h), qkv = inputs(args.workload)
+    case = Case(bsa, wl, H, qkv, args.call, knob(args), args.causal, args.plan_reuse)
+    res = case.time(K, Wm, world, local, fused=not args.no_fused)
+    plain = (args.call, knob(args), args.causal) == ("topk", 0.5, False)
+    traffic = recorded_traffic(wl.name if not args.heads else f"{wl.name}-h{H}") if plain else None
+    line = case_line(case, res, world, K, Wm, peaks, kind, traffic)
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.call == "topk" and args.plan_reuse == 1:
+        q, k, v = qkv
         qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
         op = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
         qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        stream = torch.cuda.current_stream()
 
         def e2e_step():
             # One C-ABI call on the pinned host buffers: head chunks are copied in,
             # computed and copied out as a pipeline; it returns when out is on the host.
-            bsa.sparse_attn_topk_host(qp, kp, vp, args.topk, out_host=op,
-                                      device_buffers=(qd, kd, vd, out), workspace=ws)
+            bsa.sparse_attn_topk_host(qp, kp, vp, args.topk, args.causal, out_host=op,
+                                      device_buffers=(qd, kd, vd, case.out), workspace=case.ws)
 
         for _ in range(2):
             e2e_step()
@@ -366,45 +564,22 @@ def run_b200(args, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
+        bsa.last_device_status(case.ws)
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world)
         nbytes = q.numel() * 2
-        e2e = {"value": world * dense_flops / t_e2e / 1e12, "unit": UNIT,
+        e2e = {"value": world * dense_flops(wl, H, args.causal) / t_e2e / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "ms_per_step": t_e2e * 1e3,
                "api": "sparse_attn_topk_host (pinned host q/k/v/out; copies pipelined over head chunks)"}
-
-    peaks, kind = load_peaks()
-    achieved = kept_flops / attn_s / 1e12
-    sel_bytes = 2 * B * H * N * d * 2 + B * H * wl.Qb * wl.Kb + 2 * int(mask.sum().item())
-    roofline = {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": recorded_traffic(wl.name if not args.heads else f"{wl.name}-h{H}"),
-                "peak_kind": f"bf16 dense burst, of {kind}",
-                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
-                "algorithmic_flops_per_launch": kept_flops, "avg_launch_ms": attn_s * 1e3}
-    roofline_select = {"bound": "hbm", "kernel": "pool_kernel + dots_kernel + select_kernel",
-                       "achieved": sel_bytes / sel_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                       "frac": sel_bytes / sel_s / 1e9 / peaks["hbm_gbs"],
-                       "algorithmic_bytes_per_call": sel_bytes, "avg_call_ms": sel_s * 1e3}
+    line["e2e"] = e2e
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.call == "topk" and not args.causal:
         est, desc, _ = oracle_sample(q_h, k_h, v_h, wl, args.topk, budget_s=15.0)
-        cpu = {"value": dense_flops / est / 1e12, "unit": UNIT, "cores": blas_threads(),
-               "kind": "oracle", "sample": desc}
-
+        cpu = {"value": dense_flops(wl, H, False) / est / 1e12, "unit": UNIT, "cores": blas_threads(),
+               "kind": "oracle", "sample": desc, "extrapolated": True}
+    line["cpu_baseline"] = cpu
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": whole_job_value(dense_flops, step_max, world), "unit": UNIT,
-            "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": step_max * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(wl, args.topk, H),
-            "roofline": roofline, "roofline_select": roofline_select, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 4 * K, "clocks": clk,  # pool, dots, select, attention
-            "breakdown": {"select_ms": sel_s * 1e3, "attention_ms": attn_s * 1e3,
-                          "fused_call_ms": fused_ms, "density": density,
-                          "kept_tflop": kept_flops / 1e12, "dense_tflop": dense_flops / 1e12},
-        }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
