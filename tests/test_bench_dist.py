@@ -114,3 +114,29 @@ def test_clock_sampler_falls_back_to_the_whole_run(tmp_path):
     c.proc, c.path = _DoneProc(), str(tmp_path / "smi.csv")
     rec = c.stop(t0.timestamp(), (t0 + timedelta(seconds=1)).timestamp())
     assert rec["window"] == "whole run" and rec["samples"] == 1 and rec["sm_mhz"] == 1400.0
+
+
+def test_roofline_arithmetic_of_a_bench_line():
+    """The bench line's rooflines for the Wan2.1-14B shape at density 0.5, worked by
+    hand: kept FLOPs 4 B H N^2 d rho; selection bytes 2 B H N d 2 (q, k) + B H Qb Kb
+    (mask) + 2 per kept block (idx); its sequential floor adds the dot products'
+    2 B H Qb Kb d FLOPs at 148 x 128 x 2 FLOPs per clock."""
+    import types
+
+    wl = bench.W.WORKLOADS["wan14b"]
+    B, H, N, d, Qb, Kb = 1, 40, 75600, 128, 591, 1182
+    kept = 40 * 591 * 591  # blocks kept at topk 0.5
+    case = types.SimpleNamespace(wl=wl, H=H, call="topk", mask=None)
+    res = {"density": 0.5, "attn_s": 0.05, "sel_s": 0.001, "kept": kept}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1300.0, "sm_max_mhz": 2000.0}
+    roof, kept_flops, sel = bench.rooflines(case, res, peaks, "measured", None)
+    assert kept_flops == pytest.approx(4 * B * H * N * N * d * 0.5)
+    assert roof["achieved"] == pytest.approx(kept_flops / 0.05 / 1e12)
+    assert roof["frac"] == pytest.approx(kept_flops / 0.05 / 1e12 / 1600.0)
+    sel_bytes = 2 * B * H * N * d * 2 + B * H * Qb * Kb + 2 * kept
+    assert sel["algorithmic_bytes_per_call"] == sel_bytes
+    assert sel["frac"] == pytest.approx(sel_bytes / 0.001 / 1e9 / 6000.0)
+    floor = sel_bytes / 6000e9 + 2 * B * H * Qb * Kb * d / (148 * 128 * 2 * 2000e6)
+    assert sel["sequential_floor_ms"] == pytest.approx(floor * 1e3)
+    assert sel["frac_of_sequential_floor"] == pytest.approx(floor / 0.001)
+    assert bench.dense_flops(wl, H, causal=True) == pytest.approx(4 * B * H * d * N * (N + 1) / 2)
