@@ -77,6 +77,8 @@ def parse_args():
     p.add_argument("--plan-reuse", type=int, default=1,
                    help="applies of each selection's plan per step (amortised per call)")
     p.add_argument("--sweep", action="store_true", help="one line per row of the workload table")
+    p.add_argument("--table", metavar="JSONL", default=None,
+                   help="print the markdown table of a --sweep output file (no GPU work)")
     p.add_argument("--heads", type=int, default=0,
                    help="override H (small profiling case only; not a bench line)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -529,9 +531,19 @@ def run_b200(args, world, rank, local):
                 cur = inputs(name)
             wl, H, _, qkv = cur
             case = Case(bsa, wl, H, qkv, call, param, causal, reuse)
-            res = case.time(K, Wm, world, local, fused=reuse == 1)
+            # At least ~1 s of timed steps per row, so that short calls still get
+            # clock samples (nvidia-smi samples every 50 ms); at most 500 steps.
+            t0 = time.time()
+            case.select()
+            for _ in range(reuse):
+                case.apply()
+            torch.cuda.synchronize()
+            step_est = max(time.time() - t0, 1e-4)
+            K_row = min(500, max(K, int(math.ceil(1.0 / step_est))))
+            res = case.time(K_row, Wm, world, local, fused=reuse == 1)
+            K_used = K_row
             traffic = recorded_traffic(wl.name) if (call, param, causal) == ("topk", 0.5, False) else None
-            line = case_line(case, res, world, K, Wm, peaks, kind, traffic)
+            line = case_line(case, res, world, K_used, Wm, peaks, kind, traffic)
             line["sweep"] = True
             if rank == 0:
                 print(json.dumps(line), flush=True)
@@ -598,8 +610,36 @@ def run_b200(args, world, rank, local):
     return 0
 
 
+def sweep_table(path: str) -> str:
+    """Markdown table of the JSON lines a --sweep run printed."""
+    out = ["| Config | Call | Density | Select ms | Attention ms | ms per call | Dense-eq TFLOPS | "
+           "Kept TFLOP/s | % of burst peak | % of sustained | SM MHz (median) |",
+           "|---|---|---|---|---|---|---|---|---|---|---|"]
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line.startswith("{"):
+                continue
+            d = json.loads(line)
+            c, bd, r = d["config"], d["breakdown"], d["roofline"]
+            knob = next(k for k in ("topk", "density", "threshold") if k in c)
+            call = {"topk": "top-k", "density": "caller mask p", "threshold": "cdfthreshd"}[knob]
+            call = f"{call} {c[knob]}" + (" causal" if c.get("causal") else "")
+            if c.get("plan_reuse"):
+                call += f", plan reused x{c['plan_reuse']} (amortised)"
+            clk = d.get("clocks") or {}
+            out.append(f"| {c['workload'].split(':')[0]} (B{c['B']} H{c['H']} N{c['N']} d{c['d']}) | {call} | "
+                       f"{bd['density']:.3f} | {bd['select_ms']:.3f} | {bd['attention_ms']:.3f} | "
+                       f"{bd['ms_per_call']:.3f} | {d['value']:.0f} | {r['achieved']:.0f} | "
+                       f"{100 * r['frac']:.1f} | {100 * r['frac_of_sustained']:.1f} | {clk.get('sm_mhz')} |")
+    return "\n".join(out)
+
+
 def main():
     args = parse_args()
+    if args.table:
+        print(sweep_table(args.table))
+        return 0
     world, rank, local = dist_setup()
     if args.impl == "reference":
         return run_reference(args, world, rank)

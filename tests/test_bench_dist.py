@@ -1,6 +1,7 @@
 """The benchmark's host logic on CPU: two gloo ranks, max-over-ranks timing,
 weak-scaling throughput, the reference arm's rank-0-only rule, and the clock record's
 restriction to the timed region."""
+import json
 import os
 import socket
 
@@ -140,3 +141,17 @@ def test_roofline_arithmetic_of_a_bench_line():
     assert sel["sequential_floor_ms"] == pytest.approx(floor * 1e3)
     assert sel["frac_of_sequential_floor"] == pytest.approx(floor / 0.001)
     assert bench.dense_flops(wl, H, causal=True) == pytest.approx(4 * B * H * d * N * (N + 1) / 2)
+
+
+def test_sweep_table_renders_a_line(tmp_path):
+    line = {"config": {"workload": "wan14b: Wan2.1-14B-shaped", "B": 1, "H": 40, "N": 75600, "d": 128,
+                       "topk": 0.5, "causal": True},
+            "breakdown": {"density": 0.25, "select_ms": 0.7, "attention_ms": 27.5, "ms_per_call": 28.2},
+            "value": 2074.4, "roofline": {"achieved": 1067.2, "frac": 0.663, "frac_of_sustained": 0.797},
+            "clocks": {"sm_mhz": 1500.0}}
+    p = tmp_path / "sweep.jsonl"
+    p.write_text("not json\n" + json.dumps(line) + "\n")
+    t = bench.sweep_table(str(p)).splitlines()
+    assert len(t) == 3
+    assert t[2] == ("| wan14b (B1 H40 N75600 d128) | top-k 0.5 causal | 0.250 | 0.700 | 27.500 | 28.200 | "
+                    "2074 | 1067 | 66.3 | 79.7 | 1500.0 |")
