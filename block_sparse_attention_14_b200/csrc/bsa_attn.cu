@@ -3,7 +3,11 @@
 // and its "Mask Requirements" ("SpargeAttention Documentation"): non-causal,
 // bf16 inputs, scale 1/sqrt(d).
 //
-// One CTA per (head, query block), 384 threads in three warpgroups:
+// Two kernels: bsa_fwd_kernel below (d = 128, and d = 64 when built with
+// BSA_D64_TWO_CTA=0) and bsa_fwd1_kernel (d = 64, two CTAs per SM, one softmax
+// warpgroup each; measured 5-9% faster at d = 64).
+//
+// bsa_fwd_kernel: one CTA per (head, query block), 384 threads in three warpgroups:
 //   WG0  warp 0: TMA producer for the Q tile and the kept K tiles
 //        warp 1: TMEM owner; one thread issues the Q K^T tcgen05.mma
 //        warp 2: TMA producer for the kept V tiles
@@ -559,6 +563,382 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
+// ------------------------------------------ d = 64: one softmax warpgroup per CTA
+// At d = 64 the softmax chain, not the tensor core, bounds the kernel above.
+// This variant runs TWO CTAs per SM, each with one query block, one softmax
+// warpgroup and half of the TMEM (256 columns: S at 0, O at 128, P at 192), so
+// the two softmax warpgroups of an SM are independent: each CTA has its own
+// Q K^T and P V issuers (four per SM), no cross-warpgroup merge, and one CTA's
+// prologue and epilogue overlap the other's pairs.  256 threads:
+//   warps 0-3: softmax (thread t owns query row t, TMEM lane t);
+//   warp 4: TMA producer for Q and the K tiles; warp 5: TMEM owner and Q K^T
+//   issuer; warp 6: TMA producer for the V tiles; warp 7: P V issuer.
+// Registers: launched at 128 per thread (two CTAs fill the register file);
+// setmaxnreg gives the softmax 232 and the control warps 24.
+struct Cfg1 {
+  static constexpr int D = 64;
+  static constexpr int kThreads = 256;
+  static constexpr int kChunk = 16384;             // 128 rows x 64 bf16 columns, SW128
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = 128 * D * 2;     // a pair of 64-row key blocks
+  static constexpr int kKSt = 2;
+  static constexpr int kVSt = 3;
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kKSt * kKVBytes;
+  static constexpr int kSmem = kOffV + kVSt * kKVBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColO = 128;
+  static constexpr uint32_t kColP = 192;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr unsigned kPolyPattern = BSA_POLY_PATTERN_D64;
+  static constexpr uint32_t kRegSm = 232;
+  static constexpr uint32_t kRegCtl = 24;
+  static_assert(2 * (kSmem + 1024 + 512) <= 228 * 1024, "two CTAs per SM (shared memory)");
+  static_assert(128 * kRegSm + 128 * kRegCtl <= 128 * kThreads, "register split of the launch budget");
+};
+
+template <bool kCausal>
+__global__ void __launch_bounds__(256, 2)
+    bsa_fwd1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using C = Cfg1;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[C::kKSt], bar_kempty[C::kKSt], bar_vfull[C::kVSt],
+      bar_vempty[C::kVSt], bar_sfull, bar_sfree, bar_pfull, bar_pfree, bar_odone, bar_qkdone;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_cnt;
+  __shared__ int s_tail[4];  // the last four kept key blocks (diagonal blocks are among them)
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / a.Qb;
+  const int qi = blockIdx.x - bh * a.Qb;
+  const size_t row_id = static_cast<size_t>(bh) * a.Qb + qi;
+  const int rows_valid = min(kBlockQ, a.N - qi * kBlockQ);
+  const int16_t* idx_row = a.idx + row_id * a.Kb;
+  __nv_bfloat16* out_blk = a.out + (static_cast<size_t>(bh) * a.N + static_cast<size_t>(qi) * kBlockQ) * D;
+
+  const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
+  const uint32_t sQ = base;
+  const uint32_t sK0 = base + C::kOffK;
+  const uint32_t sV0 = base + C::kOffV;
+
+  if (threadIdx.x == 0) {
+    const int c = (*reinterpret_cast<volatile uint32_t*>(&a.status->code) != 0) ? -1 : a.cnt[row_id];
+    mbar_init(smem_u32(&bar_q), 1);
+    for (int s = 0; s < C::kKSt; ++s) {
+      mbar_init(smem_u32(&bar_kfull[s]), 1);
+      mbar_init(smem_u32(&bar_kempty[s]), 1);
+    }
+    for (int s = 0; s < C::kVSt; ++s) {
+      mbar_init(smem_u32(&bar_vfull[s]), 1);
+      mbar_init(smem_u32(&bar_vempty[s]), 1);
+    }
+    mbar_init(smem_u32(&bar_sfull), 1);
+    mbar_init(smem_u32(&bar_sfree), 128);
+    mbar_init(smem_u32(&bar_pfull), 128);
+    mbar_init(smem_u32(&bar_pfree), 1);
+    mbar_init(smem_u32(&bar_odone), 1);
+    mbar_init(smem_u32(&bar_qkdone), 1);
+    fence_mbar_init();
+    s_cnt = c;
+    if (kCausal) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) s_tail[t] = (c - 4 + t >= 0) ? idx_row[c - 4 + t] : -1;
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int cnt = s_cnt;
+  if (cnt <= 0) {
+    if (cnt == 0) {  // no kept key block: the defined output is zero
+      uint4* o4 = reinterpret_cast<uint4*>(out_blk);
+      for (int e = threadIdx.x; e < rows_valid * D / 8; e += blockDim.x) o4[e] = make_uint4(0, 0, 0, 0);
+    }
+    if (warp == 5) tmem_dealloc(s_tmem, C::kTmemCols);
+    return;
+  }
+  const uint32_t tmem = s_tmem;
+  const int npairs = (cnt + 1) >> 1;
+  DeviceStatus* st = a.status;
+  const uint64_t tmo = a.timeout_ns;
+  uint32_t issued[C::kVSt] = {};
+  bool mma_issued = false;
+
+  if (warp >= 4) {
+    setmaxnreg_dec<C::kRegCtl>();
+    if ((warp == 4 || warp == 6) && lane == 0) {
+      // ---------------------------------------------- TMA producers
+      const bool is_k = warp == 4;
+      const int nst = is_k ? C::kKSt : C::kVSt;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      const uint32_t ring = is_k ? sK0 : sV0;
+      uint64_t* full = is_k ? bar_kfull : bar_vfull;
+      uint64_t* empty = is_k ? bar_kempty : bar_vempty;
+      tma_prefetch_desc(map);
+      if (is_k) {
+        tma_prefetch_desc(&tm_q);
+        mbar_expect_tx(smem_u32(&bar_q), C::kQBytes);
+        tma_load_3d(sQ, &tm_q, smem_u32(&bar_q), 0, qi * kBlockQ, bh);
+      }
+      int b0 = __ldg(idx_row), b1 = cnt > 1 ? __ldg(idx_row + 1) : 0;
+      for (int j = 0; j < npairs; ++j) {
+        const int nx0 = 2 * j + 2 < cnt ? __ldg(idx_row + 2 * j + 2) : 0;
+        const int nx1 = 2 * j + 3 < cnt ? __ldg(idx_row + 2 * j + 3) : 0;
+        const int s = j % nst;
+        const int n = j / nst;
+        if (n > 0 && !mbar_wait(smem_u32(&empty[s]), (n - 1) & 1, st, tmo, is_k ? kWaitKEmpty : kWaitVEmpty)) break;
+        const int nb = min(2, cnt - 2 * j);
+        const uint32_t bar = smem_u32(&full[s]);
+        mbar_expect_tx(bar, nb * 64 * D * 2);
+        tma_load_3d(ring + s * C::kKVBytes, map, bar, 0, b0 * kBlockK, bh);
+        if (nb == 2) tma_load_3d(ring + s * C::kKVBytes + 8192, map, bar, 0, b1 * kBlockK, bh);
+        ++issued[s];
+        b0 = nx0;
+        b1 = nx1;
+      }
+    } else if (warp == 5 && lane == 0) {
+      // ---------------------------------------------- QK^T issuer
+      const uint64_t qd = sw128_desc(sQ, 16, 1024);
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, st, tmo, kWaitQ);
+      mma_issued = true;
+      for (int j = 0; ok && j < npairs; ++j) {
+        if (j > 0 && !(ok = mbar_wait(smem_u32(&bar_sfree), (j - 1) & 1, st, tmo, kWaitSFree))) break;
+        const int s = j % C::kKSt;
+        if (!(ok = mbar_wait(smem_u32(&bar_kfull[s]), (j / C::kKSt) & 1, st, tmo, kWaitKFull))) break;
+        tc_fence_after();
+        const int nb = min(2, cnt - 2 * j);
+        const uint32_t idesc = idesc_bf16(128, 64 * nb, false);
+        const uint64_t kd = sw128_desc(sK0 + s * C::kKVBytes, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::kColS, qd + kk * 2, kd + kk * 2, idesc, kk > 0);
+        umma_commit(smem_u32(&bar_sfull));
+        umma_commit(smem_u32(&bar_kempty[s]));
+      }
+      umma_commit(smem_u32(&bar_qkdone));
+    } else if (warp == 7 && lane == 0) {
+      // ---------------------------------------------- P.V issuer
+      const uint32_t idesc_pv = idesc_bf16(128, D, true);
+      bool ok = true;
+      mma_issued = true;
+      for (int j = 0; ok && j < npairs; ++j) {
+        if (!(ok = mbar_wait(smem_u32(&bar_pfull), j & 1, st, tmo, kWaitPFull))) break;
+        const int s = j % C::kVSt;
+        if (!(ok = mbar_wait(smem_u32(&bar_vfull[s]), (j / C::kVSt) & 1, st, tmo, kWaitVFull))) break;
+        tc_fence_after();
+        const int nb = min(2, cnt - 2 * j);
+        const uint64_t vd = sw128_desc(sV0 + s * C::kKVBytes, C::kChunk, 1024);
+        const uint32_t acc0 = j >= 1 ? 1u : 0u;
+        // P: 128 lanes x 128 keys, two keys per column; 16 keys per step.
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          if (kk < nb * 4)
+            umma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, vd + kk * (2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        umma_commit(smem_u32(&bar_pfree));
+        umma_commit(smem_u32(&bar_vempty[s]));
+      }
+      umma_commit(smem_u32(&bar_odone));
+    }
+  } else {
+    setmaxnreg_inc<C::kRegSm>();
+    // ------------------------------------------------ softmax warpgroup
+    const int row = threadIdx.x;  // query row in the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t sbuf = tmem + lane_off + C::kColS;
+    const uint32_t obuf = tmem + lane_off + C::kColO;
+    const uint32_t pbuf = tmem + lane_off + C::kColP;
+    const float sl2 = a.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const int kb_last = a.Kb - 1;
+    const int tail = a.N - kb_last * kBlockK;  // valid keys in the last key block (1..64)
+    const bool ragged = tail < 64 && __ldg(idx_row + cnt - 1) == kb_last;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < npairs; ++j) {
+      ok = mbar_wait(smem_u32(&bar_sfull), j & 1, st, tmo, kWaitSFull);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const int nb = min(2, cnt - 2 * j);
+      float s[128];
+      tmem_ld128_halves(sbuf, s);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_sfree));  // the S buffer may now receive the next S
+      if (nb != 2) {
+#pragma unroll
+        for (int c = 64; c < 128; ++c) s[c] = -INFINITY;
+      }
+      if (ragged && j == npairs - 1) {
+        if (nb == 1) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = c >= tail ? -INFINITY : s[c];
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[64 + c] = c >= tail ? -INFINITY : s[64 + c];
+        }
+      }
+      if (kCausal && 2 * j + 1 >= cnt - 4) {
+        // Key column c of block b is visible to row `row` when 64 b + c <= 128 qi + row.
+        const int b0 = s_tail[2 * j - cnt + 4 < 0 ? 0 : 2 * j - cnt + 4];
+        const int b1 = nb == 2 ? s_tail[2 * j + 1 - cnt + 4] : -1;
+        const bool d0 = 2 * j - cnt + 4 >= 0 && b0 >= 2 * qi;
+        const bool d1 = b1 >= 2 * qi;
+        const int lim0 = row - (b0 - 2 * qi) * 64, lim1 = row - (b1 - 2 * qi) * 64;
+        if (d0) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = c > lim0 ? -INFINITY : s[c];
+        }
+        if (d1) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[64 + c] = c > lim1 ? -INFINITY : s[64 + c];
+        }
+      }
+      float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+      float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
+#pragma unroll
+      for (int c = 12; c < 124; c += 8) {
+        mx0 = fmax3(mx0, s[c], s[c + 1]);
+        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+      }
+      const float rmax = fmax3(fmax3(mx0, mx1, s[124]), fmax3(mx2, mx3, s[125]), fmaxf(s[126], s[127]));
+      const float m_new = fmaxf(m_run, rmax * sl2);
+      const bool need = m_new > m_run + 8.0f;  // always true for the first pair
+      const float m_use = need ? m_new : m_run;
+      const bool dead = kCausal && m_use == -INFINITY;
+      const float alpha = dead ? 1.f : ex2_approx(m_run - m_use);
+      const float m_ref = dead ? 0.f : m_use;
+      const uint64_t negm = f2_pack(-m_ref, -m_ref);
+      uint32_t pk[64];
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        if (c >= 32 && nb != 2) break;
+        const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm);
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        uint64_t pp;
+        if ((C::kPolyPattern >> (c & 7)) & 1) {
+          pp = exp2_poly2(x0, x1);
+        } else {
+          pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[c & 1] = f2_add(acc[c & 1], pp);
+        float p0, p1;
+        f2_unpack(pp, p0, p1);
+        pk[c] = pack_bf16(p0, p1);
+      }
+      float a0, a1, a2, a3;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], a2, a3);
+      l_run = l_run * alpha + ((a0 + a1) + (a2 + a3));
+      // The P tile and O are free once the previous P.V is done.
+      if (j > 0) {
+        ok = mbar_wait(smem_u32(&bar_pfree), (j - 1) & 1, st, tmo, kWaitPFree);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float o[32];
+            tmem_ld32(obuf + cc * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(obuf + cc * 32, reinterpret_cast<const uint32_t*>(o));
+          }
+          tmem_wait_st();
+        }
+      }
+      tmem_st32(pbuf, pk);
+      if (nb == 2) tmem_st32(pbuf + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_pfull));
+      m_run = m_use;
+    }
+    // ---------------------------------------------- epilogue: O / l
+    if (ok) {
+      ok = mbar_wait(smem_u32(&bar_odone), 0, st, tmo, kWaitODone);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      // m = -inf: the row saw no visible key (causal); its output is zero (its l
+      // is not exactly 0: the polynomial exp2 returns ~1e-38 for -inf).
+      const float inv = (m_run == -INFINITY || !(l_run > 0.f)) ? 0.f : 1.f / l_run;
+      __nv_bfloat16* orow = out_blk + static_cast<size_t>(row) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        tmem_ld32(obuf + cc * 32, o);
+        uint32_t wv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) wv[e] = pack_bf16(o[2 * e] * inv, o[2 * e + 1] * inv);
+        if (row < rows_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // As in bsa_fwd_kernel: drain the loads and MMAs that may still be in flight
+  // (bounded, at least 100 ms), then release the TMEM.
+  const uint64_t drain = tmo > 100000000ull ? tmo : 100000000ull;
+  __syncthreads();
+  if ((warp == 4 || warp == 6) && lane == 0) {
+    const int nst = (warp == 4) ? C::kKSt : C::kVSt;
+    for (int s = 0; s < nst; ++s) {
+      if (issued[s] == 0) continue;
+      const uint32_t bar = smem_u32(warp == 4 ? &bar_kfull[s] : &bar_vfull[s]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(bar, (issued[s] - 1) & 1)) {
+        if (globaltimer_ns() - t0 > drain) {
+          atomicCAS(&st->code, 0u, kDevTimeout);
+          break;
+        }
+      }
+    }
+    if (warp == 4) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(&bar_q), 0)) {
+        if (globaltimer_ns() - t0 > drain) {
+          atomicCAS(&st->code, 0u, kDevTimeout);
+          break;
+        }
+      }
+    }
+  }
+  if (warp == 5 || warp == 7) {
+    if (lane == 0 && mma_issued) {
+      const uint32_t fin = smem_u32(warp == 5 ? &bar_qkdone : &bar_odone);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(fin, 0)) {
+        if (globaltimer_ns() - t0 > drain) {
+          atomicCAS(&st->code, 0u, kDevTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------- host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -595,9 +975,27 @@ bool make_map(CUtensorMap* m, const void* ptr, int BH, int N, int D, int box_row
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The d = 64 kernel with one softmax warpgroup per CTA and two CTAs per SM
+// (bsa_fwd1_kernel); 0 selects the two-warpgroup kernel for d = 64 as well.
+#ifndef BSA_D64_TWO_CTA
+#define BSA_D64_TWO_CTA 1
+#endif
+
+template <bool kCausal>
+cudaError_t launch_one_wg(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const AttnArgs& args, int BH, cudaStream_t st) {
+  auto kern = bsa_fwd1_kernel<kCausal>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg1::kSmem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(args.Qb);
+  kern<<<grid, Cfg1::kThreads, Cfg1::kSmem, st>>>(mq, mk, mv, args);
+  return cudaGetLastError();
+}
+
 template <int D, bool kCausal>
 cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttnArgs& args, int BH, cudaStream_t st) {
+  if (D == 64 && BSA_D64_TWO_CTA) return launch_one_wg<kCausal>(mq, mk, mv, args, BH, st);
   using C = Cfg<D>;
   auto kern = bsa_fwd_kernel<D, kCausal>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
