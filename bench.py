@@ -65,7 +65,8 @@ TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "bsa_fwd_kernel_*_ncu.md")
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default: 10, or more so the timed region lasts ~1 s; at most 500)")
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--workload", default="wan14b", choices=sorted(W.WORKLOADS))
@@ -262,6 +263,8 @@ def run_reference(args, world, rank):
         return 0
     wl = W.WORKLOADS[args.workload]
     q, k, v = W.make_qkv(wl)
+    if args.steps is None:
+        args.steps = 10
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(q, k, v, wl, args.topk, per_step)
@@ -501,6 +504,26 @@ def knob(args):
     return {"topk": args.topk, "mask": args.density, "cdf": args.threshold}[args.call]
 
 
+def default_steps(case, world) -> int:
+    """Steps for ~1 s of timed work (at least 10, at most 500), from one untimed
+    step, so that short calls still get clock samples.  Every rank takes the
+    largest count, so all ranks time the same number of steps."""
+    t0 = time.time()
+    case.select()
+    for _ in range(case.R):
+        case.apply()
+    torch.cuda.synchronize()
+    step_est = max(time.time() - t0, 1e-4)
+    k = min(500, max(10, int(math.ceil(1.0 / step_est))))
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([k], dtype=torch.int64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        k = int(t.item())
+    return k
+
+
 def run_b200(args, world, rank, local):
     import block_sparse_attention_14_b200 as bsa
 
@@ -533,13 +556,7 @@ def run_b200(args, world, rank, local):
             case = Case(bsa, wl, H, qkv, call, param, causal, reuse)
             # At least ~1 s of timed steps per row, so that short calls still get
             # clock samples (nvidia-smi samples every 50 ms); at most 500 steps.
-            t0 = time.time()
-            case.select()
-            for _ in range(reuse):
-                case.apply()
-            torch.cuda.synchronize()
-            step_est = max(time.time() - t0, 1e-4)
-            K_row = min(500, max(K, int(math.ceil(1.0 / step_est))))
+            K_row = default_steps(case, world) if K is None else min(500, max(K, default_steps(case, world)))
             res = case.time(K_row, Wm, world, local, fused=reuse == 1)
             K_used = K_row
             traffic = recorded_traffic(wl.name) if (call, param, causal) == ("topk", 0.5, False) else None
@@ -556,6 +573,8 @@ def run_b200(args, world, rank, local):
 
     wl, H, (q_h, k_h, v_h), qkv = inputs(args.workload)
     case = Case(bsa, wl, H, qkv, args.call, knob(args), args.causal, args.plan_reuse)
+    if K is None:
+        K = default_steps(case, world)
     res = case.time(K, Wm, world, local, fused=not args.no_fused)
     plain = (args.call, knob(args), args.causal) == ("topk", 0.5, False)
     traffic = recorded_traffic(wl.name if not args.heads else f"{wl.name}-h{H}") if plain else None

@@ -44,13 +44,18 @@ namespace {
 
 // Column pairs c with bit (c % 8) set use the FMA-pipe exp2 polynomial; the
 // others use MUFU ex2.  Measured on B200 against 0, 1/8, 1/4, 3/8 and 1/2:
-// d = 128 is fastest with one pair in four (0x88), d = 64 with three in
-// eight (0xA8).
+// d = 128 is fastest with one pair in four (0x88), d = 64 in the two-warpgroup
+// kernel with three in eight (0xA8).  The one-warpgroup d = 64 kernel, whose two
+// CTAs on an SM exponentiate independently, is fastest with one or two pairs in
+// eight (0x80, 0x82, 0x88 within 0.5% of each other, 0xA8 2.5% slower, 0 1%).
 #ifndef BSA_POLY_PATTERN
 #define BSA_POLY_PATTERN 0x88
 #endif
 #ifndef BSA_POLY_PATTERN_D64
 #define BSA_POLY_PATTERN_D64 0xA8
+#endif
+#ifndef BSA_POLY_PATTERN_1WG
+#define BSA_POLY_PATTERN_1WG 0x88
 #endif
 
 enum WaitSite : uint32_t {
@@ -193,6 +198,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint64_t tmo = a.timeout_ns;
 
   // Stage-issue counters, used by the producers to drain in-flight copies.
+  static_assert(C::kKSt <= 4 && C::kVSt <= 4, "issued[] covers every ring stage");
   uint32_t issued[4] = {0, 0, 0, 0};
   bool mma_issued = false;
 
@@ -590,7 +596,7 @@ struct Cfg1 {
   static constexpr uint32_t kColO = 128;
   static constexpr uint32_t kColP = 192;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr unsigned kPolyPattern = BSA_POLY_PATTERN_D64;
+  static constexpr unsigned kPolyPattern = BSA_POLY_PATTERN_1WG;
   static constexpr uint32_t kRegSm = 232;
   static constexpr uint32_t kRegCtl = 24;
   static_assert(2 * (kSmem + 1024 + 512) <= 228 * 1024, "two CTAs per SM (shared memory)");
@@ -668,7 +674,8 @@ __global__ void __launch_bounds__(256, 2)
   const int npairs = (cnt + 1) >> 1;
   DeviceStatus* st = a.status;
   const uint64_t tmo = a.timeout_ns;
-  uint32_t issued[C::kVSt] = {};
+  // per ring stage, the loads issued into it (K and V share the counters)
+  uint32_t issued[C::kKSt > C::kVSt ? C::kKSt : C::kVSt] = {};
   bool mma_issued = false;
 
   if (warp >= 4) {
