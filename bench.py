@@ -59,7 +59,7 @@ UNIT = "dense-equiv TFLOPS"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 ATTN_SRCS = [os.path.join(ROOT, "block_sparse_attention_14_b200", "csrc", f)
              for f in ("bsa_attn.cu", "bsa_common.cuh")]
-TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "bsa_fwd_kernel_*_ncu.md")
+TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "bsa_fwd*_kernel_*_ncu.md")
 
 
 def parse_args():
@@ -109,7 +109,7 @@ def attn_source_hash() -> str:
 
 def recorded_traffic(workload: str):
     """Per-launch DRAM bytes of the attention kernel from a committed ncu summary
-    (profiles/bsa_fwd_kernel_*_ncu.md), valid only if it was taken on the current
+    (profiles/bsa_fwd*_kernel_*_ncu.md), valid only if it was taken on the current
     kernel source."""
     want = attn_source_hash()
     for path in sorted(glob.glob(TRAFFIC_GLOB)):
@@ -426,7 +426,9 @@ def rooflines(case, res, peaks, kind, traffic):
     B, N, d = wl.B, wl.N, wl.d
     kept_flops = 4.0 * B * H * N * N * d * res["density"]
     achieved = kept_flops / res["attn_s"] / 1e12
-    roofline = {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
+    # d = 64 runs the two-CTA-per-SM kernel, d = 128 the two-warpgroup one
+    roofline = {"bound": "tensor", "kernel": "bsa_fwd1_kernel" if d == 64 else "bsa_fwd_kernel",
+                "achieved": achieved,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                 "traffic": traffic, "peak_kind": f"bf16 dense burst, of {kind}",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
