@@ -24,6 +24,10 @@ selection followed by R applies of its plan (the AB-Attention refresh pattern),
 reporting the amortised time per call.  --sweep prints one line per row of the
 workload table (every config and mode), without the CPU and end-to-end legs.
 
+--steps K times exactly K steps; without it the bench picks enough steps for
+~1 s of timed work (10 to 500) from one untimed step, so that the clock samples
+fall inside the timed region.
+
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
 call (weak scaling, no collective on the data path); the step time is the
 maximum over ranks.  --impl reference times the fp64 CPU oracle on a bounded
