@@ -1,5 +1,5 @@
 """GPU parity at the full sizes of the five video-shaped workloads, in the same calls
-the benchmark times.  Selection masks are compared in full (bit-exact outside the
+the benchmark times (the causal ones too).  Selection masks are compared in full (bit-exact outside the
 tie band); attention outputs in full for the tiny and CogVideoX-2B shapes and on a
 fixed sample of query blocks ({0, 1, Qb/2, Qb-1} plus seeded random blocks,
 including the ragged last block) for the N = 75600 and N = 118800 shapes, whose
@@ -30,12 +30,12 @@ def _inputs(name):
 
 
 @functools.lru_cache(maxsize=4)
-def _oracle_select(name, topk):
+def _oracle_select(name, topk, causal=False):
     wl, (q, k, _), _ = _inputs(name)
-    return O.select(q, k, topk)
+    return O.select(q, k, topk, causal=causal)
 
 
-def _check_rows(out, wl, qkv_cpu, mask_np, heads, n_random, seed, extra=None, what=""):
+def _check_rows(out, wl, qkv_cpu, mask_np, heads, n_random, seed, extra=None, what="", causal=False):
     """Compare sampled query blocks of the listed heads, plus every (b, h, i) in
     `extra` (the rows whose GPU mask differs from the oracle's), with the oracle's
     attention over `mask_np`."""
@@ -53,7 +53,7 @@ def _check_rows(out, wl, qkv_cpu, mask_np, heads, n_random, seed, extra=None, wh
             qh, kh, vh = O.to_f64(q[b, h]), O.to_f64(k[b, h]), O.to_f64(v[b, h])
             for i in sorted(blocks):
                 lo, hi = 128 * i, min(wl.N, 128 * i + 128)
-                ref_all.append(O.attention_rows(qh, kh, vh, mask_np[b, h, i], i))
+                ref_all.append(O.attention_rows(qh, kh, vh, mask_np[b, h, i], i, causal=causal))
                 got_all.append(o[b, h, lo:hi].float().numpy())
     return assert_close(np.concatenate(got_all), np.concatenate(ref_all), what or wl.name)
 
@@ -62,26 +62,33 @@ def _differing(mc, mref, wl):
     return {(b, h): P.differing_blocks(mc, mref, b, h) for b in range(wl.B) for h in range(wl.H)}
 
 
-def _fused_case(name, topk, heads=None, n_random=4, full=False):
+def _fused_case(name, topk, heads=None, n_random=4, full=False, causal=False):
     wl, qkv_cpu, (q, k, v) = _inputs(name)
     ws = bsa.make_workspace(wl.B, wl.H, wl.N, wl.d)
-    out, mask = bsa.sparse_attn_topk(q, k, v, topk, return_mask=True, workspace=ws)
+    out, mask = bsa.sparse_attn_topk(q, k, v, topk, causal, return_mask=True, workspace=ws)
     bsa.last_device_status(ws)
-    mref, Pr = _oracle_select(name, topk)
-    mc = P.check_topk_mask(mask, mref, Pr, topk, what=f"{name} topk {topk}")
-    print(f"{name} topk {topk}: {mc}")
+    mref, Pr = _oracle_select(name, topk, causal)
+    what = f"{name} topk {topk}{' causal' if causal else ''}"
+    mc = P.check_topk_mask(mask, mref, Pr, topk, causal=causal, what=what)
+    print(f"{what}: {mc}")
     if full:
-        ref = O.block_sparse_attention(*qkv_cpu, mc.mask)
-        assert_close(out.float().cpu().numpy(), ref, f"{name}; {mc}")
+        ref = O.block_sparse_attention(*qkv_cpu, mc.mask, causal=causal)
+        assert_close(out.float().cpu().numpy(), ref, f"{what}; {mc}")
     else:
         heads = set(heads if heads is not None else range(wl.H))
         _check_rows(out, wl, qkv_cpu, mc.mask, heads, n_random, seed=int(topk * 1000),
-                    extra=_differing(mc, mref, wl), what=f"{name}; {mc}")
+                    extra=_differing(mc, mref, wl), what=f"{what}; {mc}", causal=causal)
     return mc
 
 
 def test_cogvideox2b_fused_topk05_full():
     _fused_case("cogvideox2b", 0.5, full=True)
+
+
+def test_cogvideox2b_fused_topk05_causal_full():
+    """The causal call of the d = 64 kernel at full size, every row: per-row top-k
+    over the eligible blocks, the diagonal masked element by element."""
+    _fused_case("cogvideox2b", 0.5, full=True, causal=True)
 
 
 @pytest.mark.parametrize("topk", [1.0, 0.5, 0.3, 0.1])
@@ -91,6 +98,10 @@ def test_wan13b_fused_topk_sweep(topk):
 
 def test_wan14b_fused_topk05():
     _fused_case("wan14b", 0.5, heads=[0, 7, 13, 21, 27, 39], n_random=6)
+
+
+def test_wan14b_fused_topk05_causal():
+    _fused_case("wan14b", 0.5, heads=[0, 13, 27, 39], n_random=6, causal=True)
 
 
 @pytest.mark.parametrize("density", [0.5, 0.1])
