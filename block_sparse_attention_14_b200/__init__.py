@@ -155,10 +155,14 @@ def workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def make_workspace(B: int, H: int, N: int, d: int, device="cuda") -> torch.Tensor:
+    """A workspace for the shape; its device status word (the first 256 bytes) starts
+    cleared, so last_device_status reports BSA_OK before any call has used it."""
     n = workspace_bytes(B, H, N, d)
     if n == 0:
         raise BsaError(1, lib().bsa_last_error_message().decode() or "shape rejected")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
 
 
 def _ws(q: torch.Tensor, workspace):

@@ -230,6 +230,7 @@ bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, f
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
   BSA_CUDA(launch_block_scores(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, p_out, st), "block-score kernel launch");
   return BSA_OK;
@@ -248,6 +249,7 @@ bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
   const int Kb = (s.N + kBlockK - 1) / kBlockK;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
   BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
                          mask_out, w.idx, w.cnt, st),
@@ -268,6 +270,7 @@ bsa_status sparse_attn_select_cdf(const void* q, const void* k, bsa_shape s, flo
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
   BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
            "cdf select kernel launch");
@@ -492,6 +495,7 @@ bsa_status block_sparse_attn_plan(const uint8_t* mask_id, bsa_shape s, int is_ca
   Workspace w;
   BSA_TRY(check_ws(s, ws, ws_bytes, &w));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_compact(mask_id, s.B * s.H, s.N, is_causal != 0, w.idx, w.cnt, st),
            "compaction kernel launch");
   return BSA_OK;

@@ -43,7 +43,9 @@
  *    touches no memory.  A failed launch returns BSA_ERR_CUDA.  Every wait
  *    inside the attention kernel is bounded in time; if one runs out the kernel
  *    records it in ws and returns early, which bsa_last_device_status reports
- *    as BSA_ERR_TIMEOUT.
+ *    as BSA_ERR_TIMEOUT.  Every call that takes ws first clears that status word
+ *    (on `stream`, before its kernels), so it always describes the latest call;
+ *    a workspace that no call has used yet holds whatever its memory held.
  */
 #ifndef BSA_H_
 #define BSA_H_

@@ -53,3 +53,32 @@ def test_check_true_raises_the_recorded_timeout(cuda_device):
         bsa.set_wait_timeout_ns(0)
     bsa.sparse_attn_topk(q, k, v, 0.5, out=out, workspace=ws, check=True)
     assert torch.equal(out, ref)
+
+
+def test_every_workspace_call_clears_the_status_word(cuda_device):
+    """The status word describes the latest call on the workspace: each call that
+    takes one clears the word before its kernels, the selection-only calls
+    included (their kernels never set it).  A word left nonzero by earlier use of
+    the memory must not be reported."""
+    wl = W.custom("st", B=1, H=2, d=64, N=3000, seed=8)
+    q, k, v = (t.cuda() for t in W.make_qkv(wl))
+    ws = bsa.make_workspace(wl.B, wl.H, wl.N, wl.d)
+    bsa.last_device_status(ws)  # a fresh workspace starts cleared
+    mask = torch.ones(wl.B, wl.H, wl.Qb, wl.Kb, dtype=torch.uint8, device="cuda")
+    calls = {
+        "sparse_attn_select": lambda: bsa.sparse_attn_select(q, k, 0.5, workspace=ws),
+        "sparse_attn_select_cdf": lambda: bsa.sparse_attn_select_cdf(q, k, 0.9, workspace=ws),
+        "sparse_attn_block_scores": lambda: bsa.sparse_attn_block_scores(q, k, workspace=ws),
+        "block_sparse_attn_plan": lambda: bsa.block_sparse_attn_plan(q, mask, workspace=ws),
+        "block_sparse_attn_apply": lambda: bsa.block_sparse_attn_apply(q, k, v, ws),
+        "block_sparse_attn_fwd": lambda: bsa.block_sparse_attn_fwd(q, k, v, mask, workspace=ws),
+        "sparse_attn_topk": lambda: bsa.sparse_attn_topk(q, k, v, 0.5, workspace=ws),
+        "sparse_attn_cdf": lambda: bsa.sparse_attn_cdf(q, k, v, 0.9, workspace=ws),
+    }
+    for name, call in calls.items():
+        ws[:256].fill_(0xC0)  # a stale nonzero word, as reused memory may hold
+        call()
+        try:
+            bsa.last_device_status(ws)
+        except bsa.BsaError as e:
+            raise AssertionError(f"{name} left the stale status word in place: {e}") from None
