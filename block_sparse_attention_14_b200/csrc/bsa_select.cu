@@ -111,13 +111,15 @@ __global__ void __launch_bounds__(256, 5) pool_kernel(const __nv_bfloat16* __res
 // register-tiled fp32 GEMM: CTA tile 64 query blocks x 256 key blocks, 256
 // threads, 8 x 8 outputs per thread; Qbar of the tile is kept transposed in
 // shared memory and Kbar passes through in 32-wide d chunks (transposed, rows
-// padded to 260 floats), so each d step costs 4 shared loads per 64 FMAs.
-constexpr int kDotQ = 64, kDotK = 256, kDotDc = 32, kDotThreads = 256;
+// padded to 260 floats), so each d step costs 4 shared loads per 64 FMAs.  The
+// chunks are double-buffered: the global loads of chunk c + 1 are in flight
+// (in registers) while chunk c is multiplied, then land in the other buffer.
+constexpr int kDotQ = 64, kDotK = 256, kDotDc = 16, kDotThreads = 256;
 constexpr int kDotKs = kDotK + 4;  // padded row of the transposed K chunk
 
 template <int D>
 constexpr size_t dots_smem() {
-  return sizeof(float) * (static_cast<size_t>(D) * kDotQ + static_cast<size_t>(kDotDc) * kDotKs);
+  return sizeof(float) * (static_cast<size_t>(D) * kDotQ + 2 * static_cast<size_t>(kDotDc) * kDotKs);
 }
 
 template <int D>
@@ -126,13 +128,38 @@ __global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __res
                                                            int Kb, int Kp, float* __restrict__ S) {
   extern __shared__ __align__(16) float dsm[];
   float* Qs = dsm;                       // [D][kDotQ]
-  float* Ks = dsm + D * kDotQ;           // [kDotDc][kDotKs]
+  float* Kbuf = dsm + D * kDotQ;         // 2 x [kDotDc][kDotKs]
   const int bh = blockIdx.z;
   const int i0 = blockIdx.y * kDotQ;
   const int j0 = blockIdx.x * kDotK;
   const int tid = threadIdx.x;
   const int ty = tid >> 5;  // query blocks i0 + 8 ty ... + 7 (warp-uniform)
   const int tx = tid & 31;  // key blocks j0 + 4 tx ... + 3 and j0 + 128 + 4 tx ... + 3
+  constexpr int kPer = kDotK * (kDotDc / 4) / kDotThreads;  // float4 loads per thread per chunk
+  float4 pre[kPer];
+  // element e = tid + t * threads of a chunk: key k = e / (kDotDc / 4), d group c4 = e % (kDotDc / 4)
+  auto load_chunk = [&](int dc) {
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = tid + t * kDotThreads;
+      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
+      pre[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + k < Kb)
+        pre[t] = __ldg(reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j0 + k) * D + dc) + c4);
+    }
+  };
+  auto store_chunk = [&](float* Ks) {
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = tid + t * kDotThreads;
+      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
+      Ks[(4 * c4 + 0) * kDotKs + k] = pre[t].x;
+      Ks[(4 * c4 + 1) * kDotKs + k] = pre[t].y;
+      Ks[(4 * c4 + 2) * kDotKs + k] = pre[t].z;
+      Ks[(4 * c4 + 3) * kDotKs + k] = pre[t].w;
+    }
+  };
+  load_chunk(0);
   for (int e = tid; e < kDotQ * (D / 4); e += kDotThreads) {
     const int q = e % kDotQ, d4 = e / kDotQ;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -142,25 +169,20 @@ __global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __res
     Qs[(4 * d4 + 2) * kDotQ + q] = v.z;
     Qs[(4 * d4 + 3) * kDotQ + q] = v.w;
   }
+  store_chunk(Kbuf);
   float acc[8][8];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-  for (int dc = 0; dc < D; dc += kDotDc) {
-    __syncthreads();  // the previous chunk is consumed (and Qs is written)
-    for (int e = tid; e < kDotK * (kDotDc / 4); e += kDotThreads) {
-      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + k < Kb)
-        v = __ldg(reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j0 + k) * D + dc) + c4);
-      Ks[(4 * c4 + 0) * kDotKs + k] = v.x;
-      Ks[(4 * c4 + 1) * kDotKs + k] = v.y;
-      Ks[(4 * c4 + 2) * kDotKs + k] = v.z;
-      Ks[(4 * c4 + 3) * kDotKs + k] = v.w;
-    }
-    __syncthreads();
-#pragma unroll 2
+  constexpr int kChunks = D / kDotDc;
+#pragma unroll 1
+  for (int c = 0; c < kChunks; ++c) {
+    __syncthreads();  // chunk c (and Qs) written; chunk c - 1's buffer no longer read
+    if (c + 1 < kChunks) load_chunk((c + 1) * kDotDc);
+    const float* Ks = Kbuf + (c & 1) * kDotDc * kDotKs;
+    const int dc = c * kDotDc;
+#pragma unroll 1
     for (int dd = 0; dd < kDotDc; ++dd) {
       const float4 qa = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty);
       const float4 qb = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty + 4);
@@ -180,6 +202,7 @@ __global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __res
         }
       }
     }
+    if (c + 1 < kChunks) store_chunk(Kbuf + ((c + 1) & 1) * kDotDc * kDotKs);
   }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
