@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(256, 5) pool_kernel(const __nv_bfloat16* __res
 // fmaf in ascending d order, rows padded to Kp = Kb rounded up to 4.  A
 // register-tiled fp32 GEMM: CTA tile 64 query blocks x 256 key blocks, 256
 // threads, 8 x 8 outputs per thread; Qbar of the tile is kept transposed in
-// shared memory and Kbar passes through in 32-wide d chunks (transposed, rows
+// shared memory and Kbar passes through in 16-wide d chunks (transposed, rows
 // padded to 260 floats), so each d step costs 4 shared loads per 64 FMAs.  The
 // chunks are double-buffered: the global loads of chunk c + 1 are in flight
 // (in registers) while chunk c is multiplied, then land in the other buffer.
