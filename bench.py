@@ -511,14 +511,17 @@ def knob(args):
 
 
 def default_steps(case, world) -> int:
-    """Steps for ~1 s of timed work (at least 10, at most 500), from one untimed
-    step, so that short calls still get clock samples.  Every rank takes the
-    largest count, so all ranks time the same number of steps."""
-    t0 = time.time()
-    case.select()
-    for _ in range(case.R):
-        case.apply()
-    torch.cuda.synchronize()
+    """Steps for ~1 s of timed work (at least 10, at most 500), from the second of
+    two untimed steps (the first pays one-time setup), so that short calls still
+    get clock samples.  Every rank takes the largest count, so all ranks time the
+    same number of steps."""
+    for rep in range(2):
+        torch.cuda.synchronize()
+        t0 = time.time()
+        case.select()
+        for _ in range(case.R):
+            case.apply()
+        torch.cuda.synchronize()
     step_est = max(time.time() - t0, 1e-4)
     k = min(500, max(10, int(math.ceil(1.0 / step_est))))
     if world > 1:
