@@ -242,12 +242,16 @@ __device__ __forceinline__ float* stage_row(const float* __restrict__ S, size_t 
 // taken of (key - kmin) from the top bit of the row's key range down, so the
 // first histogram spreads over all 256 buckets instead of the few that the
 // top byte of similar floats falls in (which serialised the shared atomics).
-__device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, uint8_t* mask_row,
+__device__ void warp_topk_row(float* row, int Kb, int kk, uint32_t* hist, uint8_t* mask_row,
                               int16_t* idx_row, int32_t* cnt_out) {
   const int lane = threadIdx.x & 31;
+  // The row's scores are replaced by the bit patterns of their keys in place
+  // (each lane reads back only the entries it wrote), so the passes below take
+  // the keys directly.
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int j = lane; j < Kb; j += 32) {
     const uint32_t u = float_key(row[j]);
+    row[j] = __uint_as_float(u);
     kmin = min(kmin, u);
     kmax = max(kmax, u);
   }
@@ -262,7 +266,7 @@ __device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, 
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
     for (int j = lane; j < Kb; j += 32) {
-      const uint32_t v = float_key(row[j]) - kmin;
+      const uint32_t v = __float_as_uint(row[j]) - kmin;
       if ((v & pmask) == prefix) atomicAdd(&hist[(v >> lo) & dmask], 1u);
     }
     __syncwarp();
@@ -309,7 +313,7 @@ __device__ void warp_topk_row(const float* row, int Kb, int kk, uint32_t* hist, 
   const unsigned lt = (1u << lane) - 1u;
   for (int base = 0; base < Kb; base += 32) {
     const int j = base + lane;
-    const uint32_t u = (j < Kb) ? float_key(row[j]) : 0u;
+    const uint32_t u = (j < Kb) ? __float_as_uint(row[j]) : 0u;
     const bool eq = (j < Kb) && (u == T);
     const unsigned eqb = __ballot_sync(0xffffffffu, eq);
     const bool keep = (j < Kb) && (u > T || (eq && eq_seen + __popc(eqb & lt) < need_eq));
