@@ -258,6 +258,7 @@ __device__ void warp_topk_row(float* row, int Kb, int kk, uint32_t* hist, uint8_
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   const int nbits = 32 - __clz(static_cast<int>(kmax - kmin));  // bits of the range (0 if flat)
+  const unsigned lt = (1u << lane) - 1u;
   uint32_t prefix = 0, pmask = 0;  // over v = key - kmin
   int remaining = kk;
   for (int hi = nbits; hi > 0;) {
@@ -286,7 +287,7 @@ __device__ void warp_topk_row(float* row, int Kb, int kk, uint32_t* hist, uint8_
     }
     const unsigned hit = __ballot_sync(0xffffffffu, incl >= static_cast<uint32_t>(remaining));
     const int src = __ffs(hit) - 1;  // first lane whose running count reaches `remaining`
-    uint32_t bucket = 0, above = 0;
+    uint32_t bucket = 0, above = 0, bcnt = 0;
     if (lane == src) {
       uint32_t run = incl - local;
 #pragma unroll
@@ -294,6 +295,7 @@ __device__ void warp_topk_row(float* row, int Kb, int kk, uint32_t* hist, uint8_
         if (run + cntb[t] >= static_cast<uint32_t>(remaining)) {
           bucket = 255 - 8 * lane - t;
           above = run;
+          bcnt = cntb[t];
           break;
         }
         run += cntb[t];
@@ -301,16 +303,52 @@ __device__ void warp_topk_row(float* row, int Kb, int kk, uint32_t* hist, uint8_
     }
     bucket = __shfl_sync(0xffffffffu, bucket, src);
     above = __shfl_sync(0xffffffffu, above, src);
+    bcnt = __shfl_sync(0xffffffffu, bcnt, src);
     remaining -= static_cast<int>(above);
     prefix |= bucket << lo;
     pmask |= dmask << lo;
     hi = lo;
     __syncwarp();
+    if (hi > 0 && bcnt <= 64) {
+      // At most 64 keys share the digits found so far: instead of more passes,
+      // gather them (into the histogram's space) and rank them directly.  The
+      // threshold is the candidate x with g(x) < remaining <= g(x) + e(x), where
+      // g and e count the candidates above and equal to x; every key above x is
+      // kept, and remaining - g(x) of the keys equal to x.
+      uint32_t* cand = hist;
+      int m = 0;
+      for (int j0 = 0; j0 < Kb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t v = (j < Kb) ? __float_as_uint(row[j]) - kmin : 0u;
+        const bool in = (j < Kb) && (v & pmask) == prefix;
+        const unsigned b = __ballot_sync(0xffffffffu, in);
+        if (in) cand[m + __popc(b & lt)] = v;
+        m += __popc(b);
+      }
+      __syncwarp();
+      const uint32_t x0 = lane < m ? cand[lane] : 0u;
+      const uint32_t x1 = lane + 32 < m ? cand[lane + 32] : 0u;
+      int g0 = 0, e0 = 0, g1 = 0, e1 = 0;
+      for (int c = 0; c < m; ++c) {
+        const uint32_t y = cand[c];
+        g0 += y > x0;
+        e0 += y == x0;
+        g1 += y > x1;
+        e1 += y == x1;
+      }
+      const unsigned h0 = __ballot_sync(0xffffffffu, lane < m && g0 < remaining && remaining <= g0 + e0);
+      const unsigned h1 = __ballot_sync(0xffffffffu, lane + 32 < m && g1 < remaining && remaining <= g1 + e1);
+      const int s0 = h0 ? __ffs(h0) - 1 : __ffs(h1) - 1;
+      const uint32_t xs = __shfl_sync(0xffffffffu, h0 ? x0 : x1, s0);
+      const int gs = __shfl_sync(0xffffffffu, h0 ? g0 : g1, s0);
+      prefix = xs;
+      remaining -= gs;
+      break;
+    }
   }
   const uint32_t T = prefix + kmin;
   const int need_eq = remaining;  // keys equal to T still to keep, lowest index first
   int eq_seen = 0, kept = 0;
-  const unsigned lt = (1u << lane) - 1u;
   for (int base = 0; base < Kb; base += 32) {
     const int j = base + lane;
     const uint32_t u = (j < Kb) ? __float_as_uint(row[j]) : 0u;
