@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
-SOURCES = ["bsa_api.cu", "bsa_select.cu", "bsa_attn.cu", "bsa_noalloc.cu", "bsa_reorder.cu"]
+SOURCES = ["bsa_api.cu", "bsa_select.cu", "bsa_dots_tc.cu", "bsa_attn.cu", "bsa_noalloc.cu", "bsa_reorder.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

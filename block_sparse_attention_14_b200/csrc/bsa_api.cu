@@ -232,7 +232,7 @@ bsa_status sparse_attn_block_scores(const void* q, const void* k, bsa_shape s, f
   const int BH = s.B * s.H;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_block_scores(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, p_out, st), "block-score kernel launch");
+  BSA_CUDA(launch_block_scores(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, p_out, w.status, st), "block-score kernel launch");
   return BSA_OK;
 }
 
@@ -252,7 +252,7 @@ bsa_status sparse_attn_select(const void* q, const void* k, bsa_shape s, float t
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
   BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
-                         mask_out, w.idx, w.cnt, st),
+                         mask_out, w.idx, w.cnt, w.status, st),
            "select kernel launch");
   return BSA_OK;
 }
@@ -272,7 +272,7 @@ bsa_status sparse_attn_select_cdf(const void* q, const void* k, bsa_shape s, flo
   const int BH = s.B * s.H;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, w.status, st),
            "cdf select kernel launch");
   return BSA_OK;
 }
@@ -296,7 +296,7 @@ bsa_status sparse_attn_cdf(const void* q, const void* k, const void* v, bsa_shap
   const int BH = s.B * s.H;
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
-  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, st),
+  BSA_CUDA(launch_select_cdf(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, threshold, mask_out, w.idx, w.cnt, w.status, st),
            "cdf select kernel launch");
   const char* why = nullptr;
   cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, 0, w.idx, w.cnt, w.status,
@@ -347,7 +347,7 @@ bsa_status sparse_attn_topk(const void* q, const void* k, const void* v, bsa_sha
   BSA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st), "status reset");
   BSA_CUDA(launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st), "pool kernel launch");
   BSA_CUDA(launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk, is_causal != 0,
-                         mask_out, w.idx, w.cnt, st),
+                         mask_out, w.idx, w.cnt, w.status, st),
            "select kernel launch");
   const char* why = nullptr;
   cudaError_t e = launch_attention(q, k, v, out, BH, s.N, s.d, is_causal != 0, w.idx, w.cnt, w.status,
@@ -466,7 +466,7 @@ bsa_status sparse_attn_topk_host(const void* q_host, const void* k_host, const v
       int32_t* cnt = w.cnt + hh * Qb;
       BSA_CUDA(launch_pool(qd + off, kd + off, bhc, s.N, s.d, qbar, kbar, r.select), "pool kernel launch");
       BSA_CUDA(launch_select(qbar, kbar, scores, bhc, bhc, s.N, s.d, kk, topk, is_causal != 0, nullptr, idx, cnt,
-                             r.select),
+                             w.status, r.select),
                "select kernel launch");
       BSA_CUDA(cudaEventRecord(e_sel, r.select), "event record");
       cudaStream_t sa = r.attn[c & 1];

@@ -1,6 +1,7 @@
 // Host-side launchers shared between the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -44,6 +45,19 @@ int max_score_heads(int B, int H, int N, int d, size_t capacity);
 // Records the message returned by bsa_last_error_message() on this thread.
 void set_last_error(const char* msg);
 
+// The driver's cuTensorMapEncodeTiled, looked up once (nullptr if unavailable).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// (a3) block dot products on the tensor cores (split TF32, fp32-like accuracy):
+// S[bh][i][j] = Qbar_i . Kbar_j, rows of padded_kb(Kb) floats.  Its waits are
+// bounded by timeout_ns and a timeout is recorded in `status`.
+cudaError_t launch_dots_tc(const float* qbar, const float* kbar, int BH, int Qb, int Kb, int d,
+                           float* S, DeviceStatus* status, uint64_t timeout_ns, cudaStream_t st);
+
 // (a1, a2) mean-pool q over 128-row blocks and k over 64-row blocks.
 cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, float* qbar,
                         float* kbar, cudaStream_t st);
@@ -51,19 +65,22 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
 // (a3, a4) block scores (into `scores`) and top-k; writes mask (optional), idx
 // and cnt.  kkeep is the kept count per row; with causal != 0 each row i
 // instead keeps ceil(topk * E_i) of its E_i = min(2i+2, Kb) eligible blocks.
+// `status` is the workspace's status word (the block dot products' bounded
+// waits record a timeout there).
 cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int score_heads, int BH,
                           int N, int d, int kkeep, float topk, int causal, uint8_t* mask_out,
-                          int16_t* idx, int32_t* cnt, cudaStream_t st);
+                          int16_t* idx, int32_t* cnt, DeviceStatus* status, cudaStream_t st);
 
 // cdfthreshd selection: the shortest score-ordered prefix reaching softmax mass
 // `threshold`; writes mask (optional), idx and cnt.
 cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int score_heads,
                               int BH, int N, int d, float threshold, uint8_t* mask_out,
-                              int16_t* idx, int32_t* cnt, cudaStream_t st);
+                              int16_t* idx, int32_t* cnt, DeviceStatus* status, cudaStream_t st);
 
 // (a3) block-score map only: p_out = softmax of the scaled block scores.
 cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int score_heads,
-                                int BH, int N, int d, float* p_out, cudaStream_t st);
+                                int BH, int N, int d, float* p_out, DeviceStatus* status,
+                                cudaStream_t st);
 
 // (a4') caller mask (NULL = all ones) -> idx and cnt; causal != 0 drops the
 // blocks past 2i+1 of row i.

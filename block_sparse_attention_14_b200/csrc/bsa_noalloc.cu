@@ -134,7 +134,7 @@ extern "C" bsa_status sparse_attn_topk_noalloc(const void* q, const void* k, con
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(DeviceStatus), st)) != cudaSuccess ||
       (e = launch_pool(q, k, BH, s.N, s.d, w.qbar, w.kbar, st)) != cudaSuccess ||
       (e = launch_select(w.qbar, w.kbar, w.scores, w.score_heads, BH, s.N, s.d, keep_count(topk, Kb), topk,
-                         causal, mask_out, w.idx, w.cnt, st)) != cudaSuccess)
+                         causal, mask_out, w.idx, w.cnt, w.status, st)) != cudaSuccess)
     return reject(BSA_ERR_CUDA, cudaGetErrorString(e));
   const char* why = nullptr;
   e = launch_attention(q, k, v, out, BH, s.N, s.d, causal, w.idx, w.cnt, w.status, wait_timeout_ns(), st,

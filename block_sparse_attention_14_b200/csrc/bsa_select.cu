@@ -569,8 +569,15 @@ size_t row_smem(int Kp, bool with_hist) {
          (with_hist ? sizeof(uint32_t) * kRowWarps * 256 : 0);
 }
 
+// BSA_DOTS_TC=1 (default): the block dot products on the tensor cores
+// (bsa_dots_tc.cu); 0: the fp32 FMA kernel above.
+#ifndef BSA_DOTS_TC
+#define BSA_DOTS_TC 1
+#endif
+
 cudaError_t launch_dots(const float* qbar, const float* kbar, int BH, int Qb, int Kb, int d,
-                        float* S, cudaStream_t st) {
+                        float* S, DeviceStatus* status, cudaStream_t st) {
+  if (BSA_DOTS_TC) return launch_dots_tc(qbar, kbar, BH, Qb, Kb, d, S, status, wait_timeout_ns(), st);
   const int Kp = padded_kb(Kb);
   dim3 grid((Kb + kDotK - 1) / kDotK, (Qb + kDotQ - 1) / kDotQ, BH);
   cudaError_t e;
@@ -611,7 +618,7 @@ cudaError_t launch_pool(const void* q, const void* k, int BH, int N, int d, floa
 // that chunk read them.  Everything is stream-ordered, so chunks reuse it.
 cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, int score_heads, int BH,
                           int N, int d, int kk, float topk, int causal, uint8_t* mask_out,
-                          int16_t* idx, int32_t* cnt, cudaStream_t st) {
+                          int16_t* idx, int32_t* cnt, DeviceStatus* status, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
@@ -623,7 +630,7 @@ cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, i
   for (int h0 = 0; h0 < BH; h0 += sh) {
     const int nh = BH - h0 < sh ? BH - h0 : sh;
     const size_t r0 = static_cast<size_t>(h0) * Qb;
-    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, status, st);
     if (e != cudaSuccess) return e;
     const int rows = nh * Qb;
     select_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
@@ -636,7 +643,7 @@ cudaError_t launch_select(const float* qbar, const float* kbar, float* scores, i
 
 cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* scores, int score_heads,
                               int BH, int N, int d, float threshold, uint8_t* mask_out,
-                              int16_t* idx, int32_t* cnt, cudaStream_t st) {
+                              int16_t* idx, int32_t* cnt, DeviceStatus* status, cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
@@ -649,7 +656,7 @@ cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* score
   for (int h0 = 0; h0 < BH; h0 += sh) {
     const int nh = BH - h0 < sh ? BH - h0 : sh;
     const size_t r0 = static_cast<size_t>(h0) * Qb;
-    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, status, st);
     if (e != cudaSuccess) return e;
     const int rows = nh * Qb;
     select_cdf_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
@@ -661,7 +668,8 @@ cudaError_t launch_select_cdf(const float* qbar, const float* kbar, float* score
 }
 
 cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* scores, int score_heads,
-                                int BH, int N, int d, float* p_out, cudaStream_t st) {
+                                int BH, int N, int d, float* p_out, DeviceStatus* status,
+                                cudaStream_t st) {
   const int Qb = (N + kBlockQ - 1) / kBlockQ;
   const int Kb = (N + kBlockK - 1) / kBlockK;
   const int Kp = padded_kb(Kb);
@@ -674,7 +682,7 @@ cudaError_t launch_block_scores(const float* qbar, const float* kbar, float* sco
   for (int h0 = 0; h0 < BH; h0 += sh) {
     const int nh = BH - h0 < sh ? BH - h0 : sh;
     const size_t r0 = static_cast<size_t>(h0) * Qb;
-    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, st);
+    e = launch_dots(qbar + r0 * d, kbar + static_cast<size_t>(h0) * Kb * d, nh, Qb, Kb, d, scores, status, st);
     if (e != cudaSuccess) return e;
     const int rows = nh * Qb;
     block_scores_kernel<<<(rows + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, smem, st>>>(
