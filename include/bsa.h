@@ -41,9 +41,9 @@
  *  - Errors: arguments are validated on the host before anything is launched;
  *    a rejected call returns BSA_ERR_INVALID_ARG or BSA_ERR_UNSUPPORTED and
  *    touches no memory.  A failed launch returns BSA_ERR_CUDA.  Every wait
- *    inside the attention kernel is bounded in time; if one runs out the kernel
- *    records it in ws and returns early, which bsa_last_device_status reports
- *    as BSA_ERR_TIMEOUT.  Every call that takes ws first clears that status word
+ *    inside the attention and block-score kernels is bounded in time; if one
+ *    runs out the kernel records it in ws and returns early, which
+ *    bsa_last_device_status reports as BSA_ERR_TIMEOUT.  Every call that takes ws first clears that status word
  *    (on `stream`, before its kernels), so it always describes the latest call;
  *    a workspace that no call has used yet holds whatever its memory held.
  */
