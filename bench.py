@@ -60,6 +60,7 @@ from block_sparse_attention_14_b200 import workloads as W  # noqa: E402
 
 METRIC = "ms/call and dense-equiv TFLOPS, Wan-14B-shaped topk=0.5, % of bf16 TC peak"
 UNIT = "dense-equiv TFLOPS"
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 / bf16 tensor-core ratio
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 ATTN_SRCS = [os.path.join(ROOT, "block_sparse_attention_14_b200", "csrc", f)
              for f in ("bsa_attn.cu", "bsa_common.cuh")]
@@ -443,19 +444,22 @@ def rooflines(case, res, peaks, kind, traffic):
         kern = "compact_kernel"
     else:
         sel_bytes = 2 * B * H * N * d * 2 + rows * wl.Kb + 2 * res["kept"]
-        kern = "pool_kernel + dots_kernel + " + ("select_cdf_kernel" if case.call == "cdf" else "select_kernel")
+        kern = "pool_kernel + dots_tc_kernel + " + ("select_cdf_kernel" if case.call == "cdf" else "select_kernel")
     roofline_select = {"bound": "hbm", "kernel": kern, "achieved": sel_bytes / res["sel_s"] / 1e9,
                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": sel_bytes / res["sel_s"] / 1e9 / peaks["hbm_gbs"],
                        "algorithmic_bytes_per_call": sel_bytes, "avg_call_ms": res["sel_s"] * 1e3}
     if case.call != "mask":
-        # The block dot products (2 B H Qb Kb d fp32 FLOPs) run after the pooling:
-        # the selection's floor is the HBM time plus their FMA time, at the fp32
-        # peak that 148 SMs x 128 FMA lanes give at the maximum SM clock.
+        # The block dot products (2 B H Qb Kb d FLOPs) run after the pooling, on
+        # the tensor cores as three TF32 products each (hi*hi + hi*lo + lo*hi): the
+        # selection's floor is the HBM time plus their tensor time at the TF32
+        # peak, taken as the measured bf16 peak x the nominal TF32 / bf16 ratio
+        # (1.1 / 2.25 PFLOP/s dense).
         dots_flops = 2.0 * B * H * wl.Qb * wl.Kb * d
-        fp32_peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6
-        floor_s = sel_bytes / (peaks["hbm_gbs"] * 1e9) + dots_flops / fp32_peak
-        roofline_select.update({"dots_fp32_flops": dots_flops, "fp32_peak_tflops_derived": fp32_peak / 1e12,
+        tf32_peak = peaks["bf16_tflops"] * 1e12 * TF32_PER_BF16
+        floor_s = sel_bytes / (peaks["hbm_gbs"] * 1e9) + 3.0 * dots_flops / tf32_peak
+        roofline_select.update({"dots_flops": dots_flops, "dots_tensor_flops": 3.0 * dots_flops,
+                                "tf32_peak_tflops_derived": tf32_peak / 1e12,
                                 "sequential_floor_ms": floor_s * 1e3,
                                 "frac_of_sequential_floor": floor_s / res["sel_s"]})
     return roofline, kept_flops, roofline_select

@@ -121,7 +121,7 @@ def test_roofline_arithmetic_of_a_bench_line():
     """The bench line's rooflines for the Wan2.1-14B shape at density 0.5, worked by
     hand: kept FLOPs 4 B H N^2 d rho; selection bytes 2 B H N d 2 (q, k) + B H Qb Kb
     (mask) + 2 per kept block (idx); its sequential floor adds the dot products'
-    2 B H Qb Kb d FLOPs at 148 x 128 x 2 FLOPs per clock."""
+    three TF32 products of 2 B H Qb Kb d FLOPs at the bf16 peak x 1.1 / 2.25."""
     import types
 
     wl = bench.W.WORKLOADS["wan14b"]
@@ -137,7 +137,7 @@ def test_roofline_arithmetic_of_a_bench_line():
     sel_bytes = 2 * B * H * N * d * 2 + B * H * Qb * Kb + 2 * kept
     assert sel["algorithmic_bytes_per_call"] == sel_bytes
     assert sel["frac"] == pytest.approx(sel_bytes / 0.001 / 1e9 / 6000.0)
-    floor = sel_bytes / 6000e9 + 2 * B * H * Qb * Kb * d / (148 * 128 * 2 * 2000e6)
+    floor = sel_bytes / 6000e9 + 3 * 2 * B * H * Qb * Kb * d / (1600e12 * 1.1 / 2.25)
     assert sel["sequential_floor_ms"] == pytest.approx(floor * 1e3)
     assert sel["frac_of_sequential_floor"] == pytest.approx(floor / 0.001)
     assert bench.dense_flops(wl, H, causal=True) == pytest.approx(4 * B * H * d * N * (N + 1) / 2)
