@@ -106,114 +106,9 @@ __global__ void __launch_bounds__(256, 5) pool_kernel(const __nv_bfloat16* __res
 }
 
 // ------------------------------------------------------------ block scores
-// S[bh][i][j] = Qbar_i . Kbar_j for every query block i and key block j, fp32
-// fmaf in ascending d order, rows padded to Kp = Kb rounded up to 4.  A
-// register-tiled fp32 GEMM: CTA tile 64 query blocks x 256 key blocks, 256
-// threads, 8 x 8 outputs per thread; Qbar of the tile is kept transposed in
-// shared memory and Kbar passes through in 16-wide d chunks (transposed, rows
-// padded to 260 floats), so each d step costs 4 shared loads per 64 FMAs.  The
-// chunks are double-buffered: the global loads of chunk c + 1 are in flight
-// (in registers) while chunk c is multiplied, then land in the other buffer.
-constexpr int kDotQ = 64, kDotK = 256, kDotDc = 16, kDotThreads = 256;
-constexpr int kDotKs = kDotK + 4;  // padded row of the transposed K chunk
-
-template <int D>
-constexpr size_t dots_smem() {
-  return sizeof(float) * (static_cast<size_t>(D) * kDotQ + 2 * static_cast<size_t>(kDotDc) * kDotKs);
-}
-
-template <int D>
-__global__ void __launch_bounds__(kDotThreads, 2) dots_kernel(const float* __restrict__ qbar,
-                                                           const float* __restrict__ kbar, int Qb,
-                                                           int Kb, int Kp, float* __restrict__ S) {
-  extern __shared__ __align__(16) float dsm[];
-  float* Qs = dsm;                       // [D][kDotQ]
-  float* Kbuf = dsm + D * kDotQ;         // 2 x [kDotDc][kDotKs]
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * kDotQ;
-  const int j0 = blockIdx.x * kDotK;
-  const int tid = threadIdx.x;
-  const int ty = tid >> 5;  // query blocks i0 + 8 ty ... + 7 (warp-uniform)
-  const int tx = tid & 31;  // key blocks j0 + 4 tx ... + 3 and j0 + 128 + 4 tx ... + 3
-  constexpr int kPer = kDotK * (kDotDc / 4) / kDotThreads;  // float4 loads per thread per chunk
-  float4 pre[kPer];
-  // element e = tid + t * threads of a chunk: key k = e / (kDotDc / 4), d group c4 = e % (kDotDc / 4)
-  auto load_chunk = [&](int dc) {
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const int e = tid + t * kDotThreads;
-      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
-      pre[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + k < Kb)
-        pre[t] = __ldg(reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * Kb + j0 + k) * D + dc) + c4);
-    }
-  };
-  auto store_chunk = [&](float* Ks) {
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const int e = tid + t * kDotThreads;
-      const int k = e / (kDotDc / 4), c4 = e % (kDotDc / 4);
-      Ks[(4 * c4 + 0) * kDotKs + k] = pre[t].x;
-      Ks[(4 * c4 + 1) * kDotKs + k] = pre[t].y;
-      Ks[(4 * c4 + 2) * kDotKs + k] = pre[t].z;
-      Ks[(4 * c4 + 3) * kDotKs + k] = pre[t].w;
-    }
-  };
-  load_chunk(0);
-  for (int e = tid; e < kDotQ * (D / 4); e += kDotThreads) {
-    const int q = e % kDotQ, d4 = e / kDotQ;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i0 + q < Qb) v = __ldg(reinterpret_cast<const float4*>(qbar + (static_cast<size_t>(bh) * Qb + i0 + q) * D) + d4);
-    Qs[(4 * d4 + 0) * kDotQ + q] = v.x;
-    Qs[(4 * d4 + 1) * kDotQ + q] = v.y;
-    Qs[(4 * d4 + 2) * kDotQ + q] = v.z;
-    Qs[(4 * d4 + 3) * kDotQ + q] = v.w;
-  }
-  store_chunk(Kbuf);
-  float acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-  constexpr int kChunks = D / kDotDc;
-#pragma unroll 1
-  for (int c = 0; c < kChunks; ++c) {
-    __syncthreads();  // chunk c (and Qs) written; chunk c - 1's buffer no longer read
-    if (c + 1 < kChunks) load_chunk((c + 1) * kDotDc);
-    const float* Ks = Kbuf + (c & 1) * kDotDc * kDotKs;
-    const int dc = c * kDotDc;
-#pragma unroll 1
-    for (int dd = 0; dd < kDotDc; ++dd) {
-      const float4 qa = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty);
-      const float4 qb = *reinterpret_cast<const float4*>(Qs + (dc + dd) * kDotQ + 8 * ty + 4);
-      const float4 ka = *reinterpret_cast<const float4*>(Ks + dd * kDotKs + 4 * tx);
-      const float4 kb = *reinterpret_cast<const float4*>(Ks + dd * kDotKs + 128 + 4 * tx);
-      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
-      // Two accumulators per packed fma.rn.f32x2: each lane is the same fmaf.
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const uint64_t q2 = f2_pack(qv[a], qv[a]);
-#pragma unroll
-        for (int b = 0; b < 8; b += 2) {
-          uint64_t c2 = f2_pack(acc[a][b], acc[a][b + 1]);
-          c2 = f2_fma(q2, f2_pack(kv[b], kv[b + 1]), c2);
-          f2_unpack(c2, acc[a][b], acc[a][b + 1]);
-        }
-      }
-    }
-    if (c + 1 < kChunks) store_chunk(Kbuf + ((c + 1) & 1) * kDotDc * kDotKs);
-  }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = i0 + 8 * ty + a;
-    if (i >= Qb) break;
-    float* out = S + (static_cast<size_t>(bh) * Qb + i) * Kp;
-    const int ja = j0 + 4 * tx, jb = j0 + 128 + 4 * tx;
-    if (ja < Kp) *reinterpret_cast<float4*>(out + ja) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-    if (jb < Kp) *reinterpret_cast<float4*>(out + jb) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
-  }
-}
+// S[bh][i][j] = Qbar_i . Kbar_j for every query block i and key block j, rows
+// padded to Kp = Kb rounded up to 4, are computed on the tensor cores by
+// launch_dots_tc (bsa_dots_tc.cu): split-TF32 products, fp32-like accuracy.
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
 // +0 and -0 map to the same key.
@@ -569,30 +464,9 @@ size_t row_smem(int Kp, bool with_hist) {
          (with_hist ? sizeof(uint32_t) * kRowWarps * 256 : 0);
 }
 
-// BSA_DOTS_TC=1 (default): the block dot products on the tensor cores
-// (bsa_dots_tc.cu); 0: the fp32 FMA kernel above.
-#ifndef BSA_DOTS_TC
-#define BSA_DOTS_TC 1
-#endif
-
 cudaError_t launch_dots(const float* qbar, const float* kbar, int BH, int Qb, int Kb, int d,
                         float* S, DeviceStatus* status, cudaStream_t st) {
-  if (BSA_DOTS_TC) return launch_dots_tc(qbar, kbar, BH, Qb, Kb, d, S, status, wait_timeout_ns(), st);
-  const int Kp = padded_kb(Kb);
-  dim3 grid((Kb + kDotK - 1) / kDotK, (Qb + kDotQ - 1) / kDotQ, BH);
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(dots_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(dots_smem<128>()));
-    if (e != cudaSuccess) return e;
-    dots_kernel<128><<<grid, kDotThreads, dots_smem<128>(), st>>>(qbar, kbar, Qb, Kb, Kp, S);
-  } else {
-    e = cudaFuncSetAttribute(dots_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(dots_smem<64>()));
-    if (e != cudaSuccess) return e;
-    dots_kernel<64><<<grid, kDotThreads, dots_smem<64>(), st>>>(qbar, kbar, Qb, Kb, Kp, S);
-  }
-  return cudaGetLastError();
+  return launch_dots_tc(qbar, kbar, BH, Qb, Kb, d, S, status, wait_timeout_ns(), st);
 }
 
 }  // namespace
