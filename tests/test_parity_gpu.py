@@ -102,6 +102,31 @@ def test_select_equals_fused_mask_and_block_scores(cuda_device):
     np.testing.assert_allclose(Pg, Pref, rtol=1e-4, atol=1e-7)
 
 
+@pytest.mark.parametrize("B,H,N,d", [(1, 3, 20000, 128), (2, 2, 17776, 64), (1, 2, 1000, 128)])
+def test_block_dot_products_match_fp64(B, H, N, d, cuda_device):
+    """The raw block dot products Qbar_i . Kbar_j that the selection ranks, read from
+    the workspace, against fp64 dot products of the oracle's pooled means: within
+    4e-6 of |Qbar_i| |Kbar_j| (fp32-like; the tensor cores compute them from a TF32
+    hi/lo split).  The shapes cover several 128 x 256 tiles with ragged edges in
+    both directions, and a single partial tile."""
+    wl = W.custom("dots", B=B, H=H, d=d, N=N, seed=N + d)
+    q, k, _ = W.make_qkv(wl)
+    Qb, Kb = O.block_counts(N)
+    ws = bsa.make_workspace(B, H, N, d)
+    bsa.sparse_attn_block_scores(q.cuda(), k.cuda(), workspace=ws)
+    bsa.last_device_status(ws)
+    r = lambda x: (x + 255) // 256 * 256
+    BH, Kp = B * H, (Kb + 3) // 4 * 4
+    o_s = 256 + r(BH * Qb * d * 4) + r(BH * Kb * d * 4)
+    S = ws[o_s:o_s + BH * Qb * Kp * 4].view(torch.float32).view(B, H, Qb, Kp)[..., :Kb].cpu().numpy()
+    qbar = O.pool_mean(O.to_f64(q), 128)
+    kbar = O.pool_mean(O.to_f64(k), 64)
+    S64 = np.einsum("bhid,bhjd->bhij", qbar, kbar)
+    norm = np.linalg.norm(qbar, axis=-1)[..., :, None] * np.linalg.norm(kbar, axis=-1)[..., None, :]
+    err = np.abs(S.astype(np.float64) - S64) / norm
+    assert err.max() <= 4e-6, f"max error {err.max():.2e} of |Qbar||Kbar|"
+
+
 def test_topk_one_equals_dense_bitwise(cuda_device):
     q, k, v = _cuda(*_qkv(1, 2, 3001, 128, seed=5))
     a = bsa.sparse_attn_topk(q, k, v, 1.0)
