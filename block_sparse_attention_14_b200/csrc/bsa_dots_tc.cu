@@ -8,7 +8,7 @@
 // hi*hi + hi*lo + lo*hi (the lo*lo term is below 2^-22 of the product).  In
 // fp32 the three products of a K = 8 step land in one fp32 accumulator in TMEM.
 // Measured against fp64 on the video-shaped workloads this is as accurate as
-// the fp32 FMA kernel (relative error ~1e-6 of |Qbar_i| |Kbar_j|, no ranking
+// fp32 FMA accumulation (relative error ~1e-6 of |Qbar_i| |Kbar_j|, no ranking
 // change outside the 1e-6 band).
 //
 // Persistent: one CTA per SM walks the tiles of 128 query blocks x 256 key

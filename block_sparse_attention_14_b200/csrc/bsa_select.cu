@@ -5,8 +5,8 @@
 // Method: "SpargeAttention Documentation" -- spas_sage2_attn_meansim_topk_cuda
 // ("meansim", "topk") and the 128 x 64 mask of its "Mask Requirements".
 // Pooling reads q and k once with 16-byte loads (HBM-bound); the block dot
-// products are a small fp32 GEMM per head (FMA-bound); the per-row kernels
-// read one score row each from L2.
+// products run on the tensor cores (bsa_dots_tc.cu); the per-row kernels read
+// one score row each from L2.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
