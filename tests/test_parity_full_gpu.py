@@ -139,6 +139,21 @@ def test_wan13b_fused_cdf09():
                 extra=_differing(mc, mref, wl), what=f"wan13b cdf; {mc}")
 
 
+def test_cogvideox2b_fused_cdf09_full():
+    """cdfthreshd at d = 64 and full CogVideoX-2B size, every row: the score-ordered
+    prefix reaching 0.9 of the block-score mass, then attention over it."""
+    wl, qkv_cpu, (q, k, v) = _inputs("cogvideox2b")
+    ws = bsa.make_workspace(wl.B, wl.H, wl.N, wl.d)
+    out, mask = bsa.sparse_attn_cdf(q, k, v, 0.9, return_mask=True, workspace=ws)
+    bsa.last_device_status(ws)
+    Pr = _oracle_select("cogvideox2b", 1.0)[1]
+    mref = O.cdf_mask(Pr, 0.9)
+    mc = P.check_cdf_mask(mask, mref, Pr, 0.9, what="cogvideox2b cdf 0.9")
+    print(f"cogvideox2b cdf 0.9: {mc}")
+    ref = O.block_sparse_attention(*qkv_cpu, mc.mask)
+    assert_close(out.float().cpu().numpy(), ref, f"cogvideox2b cdf 0.9; {mc}")
+
+
 def test_wan14b_host_buffer_call_matches_device_call():
     """The end-to-end call the benchmark times (pinned host buffers, default head
     chunking) writes exactly the bytes of the device call at full Wan2.1-14B size;
