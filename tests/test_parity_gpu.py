@@ -31,6 +31,23 @@ SHAPES = [(1, 2, 1024, 64), (1, 2, 1024, 128), (2, 3, 300, 64), (1, 2, 300, 128)
           (1, 1, 1, 64), (1, 1, 65, 128), (1, 2, 4113, 128), (1, 1, 2000, 64)]
 
 
+@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 257])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_sequences_through_the_whole_path(N, d, causal, cuda_device):
+    """The degenerate lengths through selection and attention: one key block
+    (flat top-k rows), a partial single query block, the 64- and 128-row block
+    edges; the block dot products then see tiles almost entirely past the data."""
+    B, H, topk = 1, 2, 0.5
+    q, k, v = _qkv(B, H, N, d, seed=N * 7 + d + causal)
+    out, mask = bsa.sparse_attn_topk(*_cuda(q, k, v), topk, causal, return_mask=True)
+    torch.cuda.synchronize()
+    mref, Pr = O.select(q, k, topk, causal=causal)
+    mc = P.check_topk_mask(mask, mref, Pr, topk, causal=causal, what=f"tiny N={N} d={d}")
+    ref = O.block_sparse_attention(q, k, v, mc.mask, causal=causal)
+    assert_close(out.float().cpu().numpy(), ref, f"tiny N={N} d={d} causal={causal}")
+
+
 @pytest.mark.parametrize("B,H,N,d", SHAPES)
 def test_dense_mask_none_matches_oracle(B, H, N, d, cuda_device):
     q, k, v = _qkv(B, H, N, d, seed=N + d, scale=1.5)
