@@ -48,6 +48,27 @@ def test_tiny_sequences_through_the_whole_path(N, d, causal, cuda_device):
     assert_close(out.float().cpu().numpy(), ref, f"tiny N={N} d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 257])
+@pytest.mark.parametrize("d", [64, 128])
+def test_tiny_sequences_cdf_and_caller_mask(N, d, cuda_device):
+    """The same lengths through cdfthreshd selection and through a caller's random
+    mask (compaction; empty rows included)."""
+    B, H = 1, 2
+    q, k, v = _qkv(B, H, N, d, seed=N * 11 + d)
+    out, mask = bsa.sparse_attn_cdf(*_cuda(q, k, v), 0.9, return_mask=True)
+    torch.cuda.synchronize()
+    Pr = O.select(q, k, 1.0)[1]
+    mref = O.cdf_mask(Pr, 0.9)
+    mc = P.check_cdf_mask(mask, mref, Pr, 0.9, what=f"tiny cdf N={N} d={d}")
+    assert_close(out.float().cpu().numpy(), O.block_sparse_attention(q, k, v, mc.mask), f"tiny cdf N={N} d={d}")
+    Qb, Kb = O.block_counts(N)
+    g = torch.Generator().manual_seed(N + d)
+    m = (torch.rand(B, H, Qb, Kb, generator=g) < 0.5).to(torch.uint8)
+    out2 = bsa.block_sparse_attn_fwd(*_cuda(q, k, v), m.cuda())
+    torch.cuda.synchronize()
+    assert_close(out2.float().cpu().numpy(), O.block_sparse_attention(q, k, v, m.numpy()), f"tiny mask N={N} d={d}")
+
+
 @pytest.mark.parametrize("B,H,N,d", SHAPES)
 def test_dense_mask_none_matches_oracle(B, H, N, d, cuda_device):
     q, k, v = _qkv(B, H, N, d, seed=N + d, scale=1.5)
